@@ -1,0 +1,157 @@
+/*
+ * nvfp4.h -- C ABI of the NVFP4 quantizer and the W4A4 block-scaled GEMM for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Format (web page "Tu pipeline NVFP4: meter 62 GB de modelo en 24 GB de
+ * laptop", section 2 "Qué es realmente NVFP4", box "Fundamento matemático:
+ * bitfield E2M1 y cuantización jerárquica"): every value is a 4-bit E2M1 code
+ * (1 sign, 2 exponent bits with bias 1, 1 mantissa bit; grid 0, ±0.5, ±1, ±1.5,
+ * ±2, ±3, ±4, ±6) times an E4M3 scale shared by 16 consecutive values along the
+ * row (the K / input dimension) times one FP32 scale for the whole tensor:
+ * W^ = q * s_b * s_g.
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" point to GPU global memory on the current CUDA
+ *    device; the caller allocates and owns all of it.  The library never
+ *    allocates or frees memory and keeps no pointer after a call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Calls enqueue work and return without synchronizing, except
+ *    nvfp4_read_device_error.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    failed check returns an error status and enqueues nothing.  Launch
+ *    failures return NVFP4_ERR_CUDA.
+ *  - Every device pointer must be 16-byte aligned (NVFP4_ERR_ALIGNMENT).
+ *  - Only sm_100 devices are accepted (NVFP4_ERR_UNSUPPORTED_DEVICE).
+ *  - Matrices are row-major.  BF16 is IEEE binary16-brain (8 exponent bits).
+ */
+#ifndef NVFP4_B200_H
+#define NVFP4_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,        /* NULL where a pointer is required, negative size, bad enum */
+    NVFP4_ERR_SHAPE = 2,              /* a size constraint below is not met */
+    NVFP4_ERR_ALIGNMENT = 3,          /* a device pointer or leading dimension is misaligned */
+    NVFP4_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100 */
+    NVFP4_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+    NVFP4_ERR_TIMEOUT = 6,            /* a bounded device-side wait gave up (see nvfp4_read_device_error) */
+    NVFP4_ERR_WORKSPACE = 7           /* workspace missing or smaller than the *_workspace_bytes query */
+} nvfp4_status;
+
+/* How a block's E4M3 scale is chosen.  The flags `--qformat nvfp4` and
+ * `--qformat nvfp4_mse` of the same page, section 2, box "Derivación del
+ * objetivo de optimización MSE vs Absmax":
+ *  ABSMAX: s_b = E4M3(amax_b / (6 s_g)) -- the block's largest value lands on 6;
+ *  MSE:    the candidates f * amax_b / (6 s_g), f = 0.3, 0.4, ..., 1.0, each
+ *          rounded to E4M3; keep the one with the least squared reconstruction
+ *          error sum_k (x_k - q_k s_b s_g)^2 (ties keep the larger scale). */
+typedef enum { NVFP4_SCALE_ABSMAX = 0, NVFP4_SCALE_MSE = 1 } nvfp4_scale_mode;
+
+/* Layout of the E4M3 block-scale buffer of a rows x cols tensor (nblk = cols/16).
+ *  SWIZZLED: the 128 x 4 tiled layout that the tcgen05 block-scaled MMA reads
+ *            (rows padded to 128, block columns padded to 4, padding zero):
+ *            byte (r, c) at ((r/128)*(Cp/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4,
+ *            Cp = ceil(nblk/4)*4.  Required by nvfp4_gemm.
+ *  LINEAR:   (rows, nblk) row-major, the checkpoint layout of the page "NVFP4 en
+ *            difusión: la misma cuantización, un motor completamente distinto",
+ *            section 2 (weight_scale of shape (out, in // 16), float8_e4m3fn). */
+typedef enum { NVFP4_SF_SWIZZLED = 0, NVFP4_SF_LINEAR = 1 } nvfp4_sf_layout;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *nvfp4_status_string(nvfp4_status status);
+
+/* NVFP4_OK when the current CUDA device is an sm_100 GPU. */
+nvfp4_status nvfp4_check_device(void);
+
+/* Bytes of the packed code buffer of a rows x cols tensor: rows * cols / 2.
+ * Two codes per byte, element 2j in bits 3:0 and element 2j+1 in bits 7:4
+ * (the (out, in // 2) uint8 buffer of "NVFP4 en difusión ...", section 2). */
+size_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of the scale buffer in the given layout (SWIZZLED includes padding). */
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout);
+
+/* Workspace nvfp4_quantize needs (device memory, any content on entry; the
+ * call overwrites it).  Constant: 256 bytes. */
+size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t cols);
+
+/* Quantize a BF16 matrix to NVFP4.
+ *   x            device, BF16, rows x cols, row stride ld_x elements (ld_x >= cols, ld_x % 8 == 0).
+ *   rows, cols   rows >= 0, cols % 16 == 0 (one scale per 16 values along a row).
+ *   mode         NVFP4_SCALE_ABSMAX or NVFP4_SCALE_MSE.
+ *   layout       layout of `scales`.
+ *   global_scale_in  device float or NULL.  NULL: s_g = amax(|x|) / 2688 (an
+ *                all-zero tensor gets 1.0), computed on the device by a first
+ *                pass over x.  Non-NULL: use *global_scale_in (> 0) and skip
+ *                that pass.
+ *   codes        device, nvfp4_codes_bytes(rows, cols) bytes, dense (row stride cols/2).
+ *   scales       device, nvfp4_scales_bytes(rows, cols, layout) bytes; every byte
+ *                is written, padding included.
+ *   global_scale_out device float or NULL: receives s_g.
+ *   block_err    device float[rows * cols/16] or NULL: the squared error
+ *                sum_k (x_k - q_k s_b s_g)^2 of each block, row-major (rows, cols/16).
+ *   workspace    device, >= nvfp4_quantize_workspace_bytes(); may be NULL only
+ *                when global_scale_in is non-NULL.
+ * Codes and scales are a deterministic function of x and s_g (bit-exact with
+ * the CPU definition shipped with the tests).  Errors: INVALID_ARG, SHAPE,
+ * ALIGNMENT, WORKSPACE, UNSUPPORTED_DEVICE, CUDA. */
+nvfp4_status nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                            nvfp4_scale_mode mode, nvfp4_sf_layout layout,
+                            const float *global_scale_in, uint8_t *codes, uint8_t *scales,
+                            float *global_scale_out, float *block_err, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* Reconstruct BF16 values W^ = q * s_b * s_g (same page, same box), evaluated as
+ * RN32(q * RN32(s_b * s_g)) and rounded to BF16 (round-to-nearest-even).
+ *   codes, scales  device, as written by nvfp4_quantize with `layout`.
+ *   global_scale   device float (s_g).
+ *   out            device BF16, rows x cols, row stride ld_out elements (ld_out % 8 == 0).
+ * Errors: INVALID_ARG, SHAPE (cols % 16), ALIGNMENT, UNSUPPORTED_DEVICE, CUDA. */
+nvfp4_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, nvfp4_sf_layout layout,
+                              const float *global_scale, int64_t rows, int64_t cols, void *out,
+                              int64_t ld_out, void *stream);
+
+/* Workspace nvfp4_gemm needs (device memory, any content on entry). */
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Block-scaled W4A4 GEMM, C = (A s_a)(B s_b)^T * s_gA * s_gB, FP32 accumulation,
+ * BF16 output ("NVFP4 en difusión ...", section 2: out = (A·s_a)(B·s_b)ᵀ with the
+ * scales applied per block inside the kernel and out_dtype BF16).
+ *   A: M x K activations -- a_codes (M, K/2) bytes, a_scales SWIZZLED for (M, K/16),
+ *      a_global_scale device float.
+ *   B: N x K weights (out x in, the checkpoint orientation) -- b_codes (N, K/2),
+ *      b_scales SWIZZLED for (N, K/16), b_global_scale device float.
+ *   C: device BF16, M x N, row stride ldc elements (ldc >= N, ldc % 8 == 0).
+ *   M, N >= 1; K >= 32 and K % 32 == 0.
+ *   workspace: device, >= nvfp4_gemm_workspace_bytes(M, N, K) bytes; holds the
+ *      status word that bounded device-side waits write on a timeout.
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, WORKSPACE, UNSUPPORTED_DEVICE, CUDA. */
+nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_global_scale,
+                        int64_t M, const uint8_t *b_codes, const uint8_t *b_scales,
+                        const float *b_global_scale, int64_t N, int64_t K, void *c, int64_t ldc,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronize `stream` and read the device status word at the start of a GEMM
+ * workspace.  Returns NVFP4_OK when no bounded wait gave up, NVFP4_ERR_TIMEOUT
+ * otherwise (and stores the raw word, which names the wait, in *word if non-NULL),
+ * NVFP4_ERR_CUDA if the copy fails.  Clears nothing: a workspace is reset by the
+ * next nvfp4_gemm that uses it. */
+nvfp4_status nvfp4_read_device_error(const void *workspace, void *stream, uint32_t *word);
+
+/* Number of kernels the most recent nvfp4_quantize / nvfp4_dequantize /
+ * nvfp4_gemm call on the calling host thread enqueued (library bookkeeping for
+ * launch counting; no counterpart on the pages). */
+int nvfp4_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_B200_H */

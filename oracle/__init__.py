@@ -89,9 +89,9 @@ def _load():
     lib.ora_dequantize.argtypes = [P, P, F, I64, I64, P]
     lib.ora_dequantize.restype = None
     lib.ora_gemm_f64.argtypes = [P, P, F, I64, P, P, F, I64, I64, P, P]
-    lib.ora_gemm_f64.restype = None
+    lib.ora_gemm_f64.restype = ctypes.c_int
     lib.ora_gemm_f64_at.argtypes = [P, P, F, P, P, F, I64, P, P, I64, P, P]
-    lib.ora_gemm_f64_at.restype = None
+    lib.ora_gemm_f64_at.restype = ctypes.c_int
     lib.ora_e2m1_encode_mag_array.argtypes = [P, I64, P]
     lib.ora_e2m1_encode_mag_array.restype = None
     lib.ora_e4m3_encode_array.argtypes = [P, I64, P]
@@ -247,8 +247,10 @@ def gemm_f64(a_codes, a_scales, a_sg, b_codes, b_scales, b_sg):
     assert b_codes.shape[1] * 2 == K
     out = np.empty((M, N), np.float64)
     absum = np.empty((M, N), np.float64)
-    _load().ora_gemm_f64(_ptr(a_codes), _ptr(a_scales), float(np.float32(a_sg)), M, _ptr(b_codes),
-                         _ptr(b_scales), float(np.float32(b_sg)), N, K, _ptr(out), _ptr(absum))
+    rc = _load().ora_gemm_f64(_ptr(a_codes), _ptr(a_scales), float(np.float32(a_sg)), M, _ptr(b_codes),
+                              _ptr(b_scales), float(np.float32(b_sg)), N, K, _ptr(out), _ptr(absum))
+    if rc != 0:
+        raise MemoryError("oracle GEMM work buffer")
     return out, absum
 
 
@@ -264,9 +266,11 @@ def gemm_f64_at(a_codes, a_scales, a_sg, b_codes, b_scales, b_sg, m_idx, n_idx):
     assert m_idx.shape == n_idx.shape
     out = np.empty(m_idx.shape, np.float64)
     absum = np.empty(m_idx.shape, np.float64)
-    _load().ora_gemm_f64_at(_ptr(a_codes), _ptr(a_scales), float(np.float32(a_sg)), _ptr(b_codes),
-                            _ptr(b_scales), float(np.float32(b_sg)), K, _ptr(m_idx), _ptr(n_idx),
-                            m_idx.size, _ptr(out), _ptr(absum))
+    rc = _load().ora_gemm_f64_at(_ptr(a_codes), _ptr(a_scales), float(np.float32(a_sg)), _ptr(b_codes),
+                                 _ptr(b_scales), float(np.float32(b_sg)), K, _ptr(m_idx), _ptr(n_idx),
+                                 m_idx.size, _ptr(out), _ptr(absum))
+    if rc != 0:
+        raise MemoryError("oracle GEMM work buffer")
     return out, absum
 
 

@@ -52,6 +52,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* ------------------------------------------------------------------------- */
@@ -354,25 +355,33 @@ void ora_dequantize(const uint8_t *codes, const uint8_t *scales, float sg, int64
 /* applied per 16-block along K, both global scales applied, in binary64.      */
 /* A is M x K (codes M x K/2, linear scales M x K/16), B is N x K likewise.    */
 /* out[m,n] = sum_k a[m,k] b[n,k]; absum[m,n] = sum_k |a[m,k] b[n,k]|.          */
-/* Every operand value q * dec(s) * s_g is exact in binary64.                  */
+/* Every operand value q * dec(s) * s_g is exact in binary64; the products are */
+/* summed in k order.                                                          */
 /* ------------------------------------------------------------------------- */
 
-static double operand_value(const uint8_t *codes, const uint8_t *scales, double sg, int64_t row,
-                            int64_t k, int64_t K)
+/* Row `row` of an operand as float64 values q * dec(s_b) * s_g (each exact). */
+static void decode_row(const uint8_t *codes, const uint8_t *scales, double sg, int64_t row, int64_t K,
+                       double *out)
 {
-    uint8_t byte = codes[row * (K / 2) + k / 2];
-    uint8_t code = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
-    return ora_e2m1_decode(code) * ora_e4m3_decode(scales[row * (K / 16) + k / 16]) * sg;
+    double e2m1[16];
+    for (int c = 0; c < 16; c++)
+        e2m1[c] = ora_e2m1_decode((uint8_t)c);
+    e4m3_table_init();
+    for (int64_t k = 0; k < K; k++) {
+        uint8_t byte = codes[row * (K / 2) + k / 2];
+        uint8_t code = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+        uint8_t s = scales[row * (K / 16) + k / 16];
+        double dec_s = (s & 0x80) ? -e4m3_table[s & 0x7F] : e4m3_table[s];
+        out[k] = e2m1[code] * dec_s * sg;
+    }
 }
 
-static void gemm_one(const uint8_t *a_codes, const uint8_t *a_scales, double a_sg,
-                     const uint8_t *b_codes, const uint8_t *b_scales, double b_sg, int64_t K,
-                     int64_t m, int64_t n, double *out, double *absum)
+/* out = sum_k a[k] b[k] in k order; absum = sum_k |a[k] b[k]|. */
+static void dot_f64(const double *a, const double *b, int64_t K, double *out, double *absum)
 {
     double acc = 0.0, mag = 0.0;
     for (int64_t k = 0; k < K; k++) {
-        double p = operand_value(a_codes, a_scales, a_sg, m, k, K) *
-                   operand_value(b_codes, b_scales, b_sg, n, k, K);
+        double p = a[k] * b[k];
         acc += p;
         mag += fabs(p);
     }
@@ -381,25 +390,43 @@ static void gemm_one(const uint8_t *a_codes, const uint8_t *a_scales, double a_s
         *absum = mag;
 }
 
-void ora_gemm_f64(const uint8_t *a_codes, const uint8_t *a_scales, float a_sg, int64_t M,
-                  const uint8_t *b_codes, const uint8_t *b_scales, float b_sg, int64_t N,
-                  int64_t K, double *out, double *absum)
+/* Returns 0, or -1 when a work buffer cannot be allocated. */
+int ora_gemm_f64(const uint8_t *a_codes, const uint8_t *a_scales, float a_sg, int64_t M,
+                 const uint8_t *b_codes, const uint8_t *b_scales, float b_sg, int64_t N, int64_t K,
+                 double *out, double *absum)
 {
+    double *a = (double *)malloc(sizeof(double) * (size_t)(M * K + K));
+    if (!a)
+        return -1;
+    double *b = a + M * K;
     for (int64_t m = 0; m < M; m++)
-        for (int64_t n = 0; n < N; n++)
-            gemm_one(a_codes, a_scales, a_sg, b_codes, b_scales, b_sg, K, m, n, &out[m * N + n],
-                     absum ? &absum[m * N + n] : NULL);
+        decode_row(a_codes, a_scales, a_sg, m, K, a + m * K);
+    for (int64_t n = 0; n < N; n++) {
+        decode_row(b_codes, b_scales, b_sg, n, K, b);
+        for (int64_t m = 0; m < M; m++)
+            dot_f64(a + m * K, b, K, &out[m * N + n], absum ? &absum[m * N + n] : NULL);
+    }
+    free(a);
+    return 0;
 }
 
 /* The same reference at `count` sampled positions (m_idx[i], n_idx[i]). */
-void ora_gemm_f64_at(const uint8_t *a_codes, const uint8_t *a_scales, float a_sg,
-                     const uint8_t *b_codes, const uint8_t *b_scales, float b_sg, int64_t K,
-                     const int64_t *m_idx, const int64_t *n_idx, int64_t count, double *out,
-                     double *absum)
+int ora_gemm_f64_at(const uint8_t *a_codes, const uint8_t *a_scales, float a_sg,
+                    const uint8_t *b_codes, const uint8_t *b_scales, float b_sg, int64_t K,
+                    const int64_t *m_idx, const int64_t *n_idx, int64_t count, double *out,
+                    double *absum)
 {
-    for (int64_t i = 0; i < count; i++)
-        gemm_one(a_codes, a_scales, a_sg, b_codes, b_scales, b_sg, K, m_idx[i], n_idx[i], &out[i],
-                 absum ? &absum[i] : NULL);
+    double *a = (double *)malloc(sizeof(double) * (size_t)(2 * K));
+    if (!a)
+        return -1;
+    double *b = a + K;
+    for (int64_t i = 0; i < count; i++) {
+        decode_row(a_codes, a_scales, a_sg, m_idx[i], K, a);
+        decode_row(b_codes, b_scales, b_sg, n_idx[i], K, b);
+        dot_f64(a, b, K, &out[i], absum ? &absum[i] : NULL);
+    }
+    free(a);
+    return 0;
 }
 
 /* ------------------------------------------------------------------------- */

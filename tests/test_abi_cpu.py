@@ -1,0 +1,107 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every symbol the
+header declares, and its host-side logic (size queries, argument validation)
+answers before any CUDA call.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a4_gemm_quantize_b200 as nv
+from w4a4_gemm_quantize_b200 import build as nvbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nvbuild.build()
+    return nv.load_library()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in nv.SIGNATURES, f"binding lacks {n}"
+    assert set(nv.SIGNATURES) == set(names)
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        s = lib.nvfp4_status_string(code)
+        assert s and s != b"unknown status"
+    assert lib.nvfp4_status_string(99) == b"unknown status"
+
+
+def test_size_queries(lib):
+    assert lib.nvfp4_codes_bytes(4096, 4096) == 4096 * 2048
+    assert lib.nvfp4_scales_bytes(4096, 4096, nv.SF_LINEAR) == 4096 * 256
+    assert lib.nvfp4_scales_bytes(4096, 4096, nv.SF_SWIZZLED) == 4096 * 256
+    assert lib.nvfp4_scales_bytes(130, 48, nv.SF_SWIZZLED) == 256 * 4   # rows -> 256, 3 blocks -> 4
+    assert lib.nvfp4_scales_bytes(1, 16, nv.SF_SWIZZLED) == 128 * 4
+    assert lib.nvfp4_quantize_workspace_bytes(1, 16) >= 4
+    assert lib.nvfp4_gemm_workspace_bytes(1, 1, 32) >= 4
+    assert lib.nvfp4_codes_bytes(-1, 16) == 0
+
+
+def _q(lib, x=16, rows=4, cols=32, ld=32, mode=0, layout=0, gs=None, codes=16, scales=16, ws=16,
+       ws_bytes=256):
+    P = ctypes.c_void_p
+    return lib.nvfp4_quantize(P(x) if x else None, rows, cols, ld, mode, layout, P(gs) if gs else None,
+                              P(codes) if codes else None, P(scales) if scales else None, None, None,
+                              P(ws) if ws else None, ws_bytes, None)
+
+
+def test_quantize_validation_before_any_cuda_call(lib):
+    assert _q(lib, cols=24, ld=24) == 2            # cols % 16
+    assert _q(lib, rows=-1) == 1                    # negative size
+    assert _q(lib, ld=16) == 1                      # ld < cols
+    assert _q(lib, mode=5) == 1                     # unknown mode
+    assert _q(lib, layout=7) == 1                   # unknown layout
+    assert _q(lib, x=0) == 1                        # NULL input
+    assert _q(lib, ws=0) == 7                       # no workspace, no global scale
+    assert _q(lib, ws_bytes=3) == 7                 # workspace too small
+    assert _q(lib, x=8) == 3                        # misaligned input
+    assert _q(lib, codes=24) == 3                   # misaligned output
+    assert _q(lib, ld=36) == 3                      # row stride not 16-byte aligned
+    # everything valid: the device check runs and fails without a GPU
+    assert _q(lib) in (4, 5)
+
+
+def test_gemm_validation_before_any_cuda_call(lib):
+    P = ctypes.c_void_p
+
+    def g(M=16, N=16, K=64, ldc=16, ptr=16, ws=16, ws_bytes=256, gs=16):
+        p = P(ptr) if ptr else None
+        return lib.nvfp4_gemm(p, p, P(gs), M, p, p, P(gs), N, K, p, ldc, P(ws) if ws else None, ws_bytes, None)
+
+    assert g(K=48) == 2          # K % 32
+    assert g(M=0) == 1
+    assert g(ldc=8) == 1         # ldc < N
+    assert g(ptr=0) == 1
+    assert g(ws=0) == 7
+    assert g(ptr=8) == 3
+    assert g(ldc=20) == 3
+    assert g(gs=2) == 3
+    assert g() in (4, 5)
+
+
+def test_dequantize_validation(lib):
+    P = ctypes.c_void_p
+    assert lib.nvfp4_dequantize(P(16), P(16), 0, P(16), 4, 24, P(16), 24, None) == 2
+    assert lib.nvfp4_dequantize(P(16), P(16), 0, P(16), 0, 32, P(16), 32, None) == 0  # empty: nothing to do
+    assert lib.nvfp4_dequantize(None, P(16), 0, P(16), 4, 32, P(16), 32, None) == 1
+    assert lib.nvfp4_dequantize(P(16), P(16), 0, P(16), 4, 32, P(24), 32, None) == 3
+
+
+def test_read_device_error_needs_workspace(lib):
+    assert lib.nvfp4_read_device_error(None, None, None) == 1

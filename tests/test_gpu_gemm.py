@@ -1,0 +1,157 @@
+"""GPU parity of the W4A4 GEMM against the oracle's float64 reference.
+
+Operands are quantized by the oracle (so these tests do not lean on the GPU
+quantizer) and uploaded; C = (A s_a)(B s_b)^T s_gA s_gB comes back in BF16.
+
+Tolerance (per element): |C - ref| <= 1e-3 * S + 1e-6 + 2^-8 |ref|, where ref is
+the float64 dot product of the dequantized operands and S = sum_k |a_k b_k|.  The
+first two terms are the stated accumulation bound; the last is the rounding of
+the result to BF16 (8 significant bits), which the BF16 output format forces and
+which alone can exceed 1e-3 * S when one product dominates the sum.  In addition
+most elements must equal BF16_RNE(ref) exactly, which catches small systematic
+errors (a wrong scale on some blocks) that the bound would let through.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import w4a4_gemm_quantize_b200 as nv
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_operand(x_cpu, mode=oracle.SCALE_ABSMAX):
+    codes, sc, sg, _ = oracle.quantize(x_cpu, mode)
+    return codes, sc, sg
+
+
+def upload(codes, sc, sg):
+    rows, half = codes.shape
+    return nv.NVFP4Tensor(torch.from_numpy(np.ascontiguousarray(codes)).cuda(),
+                          torch.from_numpy(oracle.swizzle_scales(sc)).cuda(),
+                          torch.tensor([sg], dtype=torch.float32, device="cuda"), rows, half * 2, nv.SF_SWIZZLED)
+
+
+def check(c_gpu, ref, absum, min_exact=0.9):
+    c = c_gpu.astype(np.float64)
+    err = np.abs(c - ref)
+    bound = 1e-3 * absum + 1e-6 + np.abs(ref) * 2.0 ** -8
+    bad = err > bound
+    assert not bad.any(), (f"{bad.sum()} elements out of bound; worst excess "
+                           f"{(err - bound).max():.3e} at {np.unravel_index((err - bound).argmax(), err.shape)}")
+    rne = torch.from_numpy(ref.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    exact = np.mean(c == rne)
+    assert exact >= min_exact, f"only {exact:.3f} of the elements equal BF16(ref)"
+
+
+def run_full(a, b, M, N, K):
+    A, B = upload(*a), upload(*b)
+    out = nv.nvfp4_gemm(A, B)
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    out2 = nv.nvfp4_gemm(A, B, workspace=ws)
+    assert nv.read_device_error(ws) == 0
+    assert torch.equal(out, out2)  # deterministic
+    ref, absum = oracle.gemm_f64(*a, *b)
+    check(out.float().cpu().numpy(), ref, absum)
+    return out
+
+
+def test_pr1_reference_config(cuda_device):
+    """W4A4 GEMM M=16, N=256, K=256 on the PR1 tensors (absmax scales)."""
+    d = workloads.pr1(seed=0)
+    run_full(oracle_operand(d["x"]), oracle_operand(d["w"]), 16, 256, 256)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 64), (7, 136, 32), (128, 256, 256), (200, 320, 544),
+                                   (129, 384, 1056), (300, 520, 2080), (256, 512, 4096)])
+def test_ragged_shapes_full_compare(cuda_device, M, N, K):
+    """Several tiles in M and N, partial K-tiles (K % 256 != 0, K % 64 == 32), N not
+    a multiple of 128 (a tile whose second scale group is absent)."""
+    xa = workloads.activation(M, K, seed=M, n_outlier_channels=min(4, K // 16))
+    xb = workloads.gaussian_weight(N, K, 0.02, seed=N)
+    run_full(oracle_operand(xa), oracle_operand(xb, oracle.SCALE_MSE), M, N, K)
+
+
+def test_zero_and_sign_cases(cuda_device):
+    M, N, K = 64, 256, 256
+    z = workloads.to_bf16(np.zeros((M, K), np.float32))
+    w = workloads.gaussian_weight(N, K, 1.0, seed=3)
+    out = nv.nvfp4_gemm(upload(*oracle_operand(z)), upload(*oracle_operand(w)))
+    assert not out.float().abs().sum().item()
+    neg = workloads.to_bf16(-workloads.gaussian_weight(M, K, 1.0, seed=4).float().numpy())
+    run_full(oracle_operand(neg), oracle_operand(w), M, N, K)
+
+
+def test_integer_grid_special_case(cuda_device):
+    """All block scales 1 and s_g = 1: C is an exact integer matmul / 4."""
+    r = np.random.default_rng(12)
+    M, N, K = 130, 260, 320
+    ca = r.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    cb = r.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sa = np.full((M, K // 16), 0x38, np.uint8)
+    sb = np.full((N, K // 16), 0x38, np.uint8)
+    run_full((ca, sa, np.float32(1)), (cb, sb, np.float32(1)), M, N, K)
+
+
+def _sampled(M, N, K, a, b, out, n_samples=3000, seed=0):
+    r = np.random.default_rng(seed)
+    mi = np.concatenate([r.integers(0, M, n_samples), np.repeat(np.arange(min(M, 128)), 4),
+                         np.full(64, M - 1)])
+    ni = np.concatenate([r.integers(0, N, n_samples), r.integers(0, N, 4 * min(M, 128)),
+                         np.arange(N - 64, N)])
+    ref, absum = oracle.gemm_f64_at(*a, *b, mi, ni)
+    got = out.float().cpu().numpy()[mi, ni]
+    check(got, ref, absum)
+
+
+def test_decode_config(cuda_device):
+    """Decode linear: M in {1, 8, 32}, K=4096, N=14336 (weights pre-quantized)."""
+    w = oracle_operand(workloads.gaussian_weight(14336, 4096, 0.02, seed=0), oracle.SCALE_MSE)
+    W = upload(*w)
+    for m in (1, 8, 32):
+        x = oracle_operand(workloads.activation(m, 4096, seed=m))
+        out = nv.nvfp4_gemm(upload(*x), W)
+        ref, absum = oracle.gemm_f64(*x, *w)
+        check(out.float().cpu().numpy(), ref, absum)
+
+
+def test_prefill_config_sampled(cuda_device):
+    """Prefill linear M=4096, K=4096, N=14336 at full size, sampled outputs."""
+    M, N, K = 4096, 14336, 4096
+    a = oracle_operand(workloads.activation(M, K, seed=0))
+    b = oracle_operand(workloads.gaussian_weight(N, K, 0.02, seed=0), oracle.SCALE_ABSMAX)
+    out = nv.nvfp4_gemm(upload(*a), upload(*b))
+    _sampled(M, N, K, a, b, out)
+
+
+def test_prefill_down_projection_sampled(cuda_device):
+    """Down projection M=4096, K=14336, N=4096 (56 K-tiles)."""
+    M, N, K = 4096, 4096, 14336
+    a = oracle_operand(workloads.activation(M, K, seed=1, stream=workloads.STREAM_X2))
+    b = oracle_operand(workloads.gaussian_weight(N, K, 0.02, seed=1, stream=workloads.STREAM_W2))
+    out = nv.nvfp4_gemm(upload(*a), upload(*b))
+    _sampled(M, N, K, a, b, out, seed=1)
+
+
+def test_scaled_mm_library_pin_of_the_oracle(cuda_device):
+    """Pin the oracle's nibble order and swizzled scale layout against a library
+    routine: torch._scaled_mm (cuBLASLt NVFP4) reads the oracle's bytes and must
+    agree with the oracle's float64 GEMM."""
+    if not hasattr(torch, "float4_e2m1fn_x2"):
+        pytest.skip("torch has no float4_e2m1fn_x2")
+    M, N, K = 128, 256, 512
+    a = oracle_operand(workloads.activation(M, K, seed=9))
+    b = oracle_operand(workloads.gaussian_weight(N, K, 0.02, seed=9), oracle.SCALE_MSE)
+    A = torch.from_numpy(a[0]).cuda().view(torch.float4_e2m1fn_x2)
+    B = torch.from_numpy(b[0]).cuda().view(torch.float4_e2m1fn_x2)
+    sa = torch.from_numpy(oracle.swizzle_scales(a[1])).cuda().view(torch.float8_e4m3fn)
+    sb = torch.from_numpy(oracle.swizzle_scales(b[1])).cuda().view(torch.float8_e4m3fn)
+    try:
+        out = torch._scaled_mm(A, B.t(), scale_a=sa, scale_b=sb, out_dtype=torch.float32)
+    except (RuntimeError, TypeError) as e:
+        pytest.skip(f"torch._scaled_mm rejects NVFP4 here: {e}")
+    got = out.double().cpu().numpy() * float(a[2]) * float(b[2])
+    ref, absum = oracle.gemm_f64(*a, *b)
+    assert np.all(np.abs(got - ref) <= 1e-5 * absum + 1e-9)

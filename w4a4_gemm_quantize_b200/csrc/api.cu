@@ -1,0 +1,201 @@
+// api.cu -- the extern "C" entry points declared in include/nvfp4.h: host-side
+// validation, workspace layout and kernel launches.  No allocation, no
+// synchronisation (except nvfp4_read_device_error).
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/nvfp4.h"
+#include "internal.h"
+
+namespace nvfp4 {
+thread_local int g_last_launches = 0;
+}
+
+namespace {
+
+constexpr size_t kQuantizeWorkspace = 256;  // word 0: global amax (BF16 magnitude bits)
+constexpr size_t kGemmWorkspace = 256;      // word 0: device status word of bounded waits
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+nvfp4_status check_device_cached() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return NVFP4_ERR_CUDA;
+  static int verdict[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+  if (dev < 64 && verdict[dev] != 0) return verdict[dev] == 1 ? NVFP4_OK : NVFP4_ERR_UNSUPPORTED_DEVICE;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  const bool ok = (major == 10 && minor == 0);
+  if (dev < 64) verdict[dev] = ok ? 1 : 2;
+  return ok ? NVFP4_OK : NVFP4_ERR_UNSUPPORTED_DEVICE;
+}
+
+nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_string(nvfp4_status status) {
+  switch (status) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_SHAPE: return "unsupported shape";
+    case NVFP4_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case NVFP4_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_TIMEOUT: return "device-side wait timed out";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+nvfp4_status nvfp4_check_device(void) { return check_device_cached(); }
+
+size_t nvfp4_codes_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(cols / 2);
+}
+
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout) {
+  if (rows < 0 || cols < 0) return 0;
+  const int64_t nblk = cols / 16;
+  if (layout == NVFP4_SF_LINEAR) return static_cast<size_t>(rows * nblk);
+  const int64_t rp = (rows + 127) / 128 * 128;
+  const int64_t cp = (nblk + 3) / 4 * 4;
+  return static_cast<size_t>(rp * cp);
+}
+
+size_t nvfp4_quantize_workspace_bytes(int64_t, int64_t) { return kQuantizeWorkspace; }
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld_x, nvfp4_scale_mode mode,
+                            nvfp4_sf_layout layout, const float* global_scale_in, uint8_t* codes, uint8_t* scales,
+                            float* global_scale_out, float* block_err, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (rows < 0 || cols < 0 || ld_x < cols) return NVFP4_ERR_INVALID_ARG;
+  if (mode != NVFP4_SCALE_ABSMAX && mode != NVFP4_SCALE_MSE) return NVFP4_ERR_INVALID_ARG;
+  if (layout != NVFP4_SF_SWIZZLED && layout != NVFP4_SF_LINEAR) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return NVFP4_ERR_SHAPE;
+  if (rows == 0 || cols == 0) {
+    if (global_scale_in == nullptr && (workspace == nullptr || workspace_bytes < kQuantizeWorkspace))
+      return NVFP4_ERR_WORKSPACE;
+  }
+  if (rows > 0 && cols > 0 && (x == nullptr || codes == nullptr || scales == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if (global_scale_in == nullptr && (workspace == nullptr || workspace_bytes < kQuantizeWorkspace))
+    return NVFP4_ERR_WORKSPACE;
+  if ((x && !aligned16(x)) || (codes && !aligned16(codes)) || (scales && !aligned16(scales)) ||
+      (workspace && !aligned16(workspace)) || ld_x % 8 != 0)
+    return NVFP4_ERR_ALIGNMENT;
+  if ((global_scale_in && (reinterpret_cast<uintptr_t>(global_scale_in) & 3u)) ||
+      (global_scale_out && (reinterpret_cast<uintptr_t>(global_scale_out) & 3u)) ||
+      (block_err && (reinterpret_cast<uintptr_t>(block_err) & 3u)))
+    return NVFP4_ERR_ALIGNMENT;
+  nvfp4_status st = check_device_cached();
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const bool swz = layout == NVFP4_SF_SWIZZLED;
+  uint32_t* amax_word = static_cast<uint32_t*>(workspace);
+  if (global_scale_in == nullptr) {
+    if (cudaMemsetAsync(amax_word, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (rows > 0 && cols > 0) {
+      st = from_cuda(nvfp4::launch_amax(static_cast<const uint16_t*>(x), rows, cols, ld_x, amax_word, s));
+      if (st != NVFP4_OK) return st;
+      ++nvfp4::g_last_launches;
+    }
+  }
+  if (rows == 0 || cols == 0) {
+    // Nothing to encode; still publish s_g (1.0 for an empty tensor, or the given one).
+    if (global_scale_out) {
+      if (global_scale_in) {
+        if (cudaMemcpyAsync(global_scale_out, global_scale_in, sizeof(float), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+          return NVFP4_ERR_CUDA;
+      } else {
+        static const float one = 1.0f;
+        if (cudaMemcpyAsync(global_scale_out, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess)
+          return NVFP4_ERR_CUDA;
+      }
+    }
+    return NVFP4_OK;
+  }
+  if (swz) {
+    st = from_cuda(nvfp4::launch_sf_pad_zero(scales, rows, cols / 16, s));
+    if (st != NVFP4_OK) return st;
+    const int64_t rp = (rows + 127) / 128 * 128, cp = (cols / 16 + 3) / 4 * 4;
+    if (rp != rows || cp != cols / 16) ++nvfp4::g_last_launches;
+  }
+  st = from_cuda(nvfp4::launch_quantize(static_cast<const uint16_t*>(x), rows, cols, ld_x, static_cast<int>(mode),
+                                        swz, global_scale_in, amax_word, codes, scales, global_scale_out, block_err,
+                                        s));
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
+}
+
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, nvfp4_sf_layout layout,
+                              const float* global_scale, int64_t rows, int64_t cols, void* out, int64_t ld_out,
+                              void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (rows < 0 || cols < 0 || ld_out < cols) return NVFP4_ERR_INVALID_ARG;
+  if (layout != NVFP4_SF_SWIZZLED && layout != NVFP4_SF_LINEAR) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return NVFP4_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (!codes || !scales || !global_scale || !out) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(out) || ld_out % 8 != 0 ||
+      (reinterpret_cast<uintptr_t>(global_scale) & 3u))
+    return NVFP4_ERR_ALIGNMENT;
+  nvfp4_status st = check_device_cached();
+  if (st != NVFP4_OK) return st;
+  st = from_cuda(nvfp4::launch_dequantize(codes, scales, layout == NVFP4_SF_SWIZZLED, global_scale, rows, cols,
+                                          static_cast<uint16_t*>(out), ld_out, static_cast<cudaStream_t>(stream)));
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
+}
+
+size_t nvfp4_gemm_workspace_bytes(int64_t, int64_t, int64_t) { return kGemmWorkspace; }
+
+nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale, int64_t M,
+                        const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale, int64_t N,
+                        int64_t K, void* c, int64_t ldc, void* workspace, size_t workspace_bytes, void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (M < 1 || N < 1 || K < 1 || ldc < N) return NVFP4_ERR_INVALID_ARG;
+  if (K % 32 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return NVFP4_ERR_SHAPE;
+  if (!a_codes || !a_scales || !a_global_scale || !b_codes || !b_scales || !b_global_scale || !c)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) ||
+      !aligned16(c) || !aligned16(workspace) || ldc % 8 != 0 ||
+      (reinterpret_cast<uintptr_t>(a_global_scale) & 3u) || (reinterpret_cast<uintptr_t>(b_global_scale) & 3u))
+    return NVFP4_ERR_ALIGNMENT;
+  nvfp4_status st = check_device_cached();
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  const cudaError_t e = nvfp4::launch_gemm(a_codes, a_scales, a_global_scale, M, b_codes, b_scales, b_global_scale,
+                                           N, K, static_cast<uint16_t*>(c), ldc, status, s);
+  if (e == cudaErrorInvalidValue) return NVFP4_ERR_CUDA;
+  st = from_cuda(e);
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
+}
+
+nvfp4_status nvfp4_read_device_error(const void* workspace, void* stream, uint32_t* word) {
+  if (!workspace) return NVFP4_ERR_INVALID_ARG;
+  uint32_t w = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&w, workspace, sizeof(w), cudaMemcpyDeviceToHost, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (word) *word = w;
+  return w == 0 ? NVFP4_OK : NVFP4_ERR_TIMEOUT;
+}
+
+// Kernels the most recent call on this thread enqueued (benchmark bookkeeping).
+int nvfp4_last_launch_count(void) { return nvfp4::g_last_launches; }
+
+}  // extern "C"

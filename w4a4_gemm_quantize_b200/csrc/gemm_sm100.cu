@@ -1,0 +1,307 @@
+// gemm_sm100.cu -- block-scaled NVFP4 x NVFP4 GEMM on the sm_100a tensor cores.
+//
+// C = (A s_a)(B s_b)^T * s_gA * s_gB with FP32 accumulation and BF16 output: the
+// equation out = (A·s_a) × (B·s_b)ᵀ of the web page "NVFP4 en difusión: la
+// misma cuantización, un motor completamente distinto", section 2 "NVFP4 sin
+// vLLM: torch._scaled_mm a mano" -- the per-16 E4M3 scales travel as separate
+// tensors and are applied per block inside the kernel; the result is BF16.
+//
+// Design (one CTA per 128 x BN output tile, 6 warps):
+//   warp 4  TMA producer: per K-tile of 256 values, a 128 x 128-byte A tile and a
+//           BN x 128-byte B tile (tensor maps, 128-byte swizzle) plus the scale
+//           tiles (plain bulk copies of the 512-byte 128x4 atoms), into a
+//           STAGES-deep shared-memory ring guarded by full/empty mbarriers;
+//   warp 5  allocates TMEM and issues, from one thread, tcgen05.cp of the scale
+//           atoms into TMEM and tcgen05.mma.kind::mxf4nvf4.block_scale.block16
+//           (128 x BN x 64 per instruction) accumulating in TMEM; tcgen05.commit
+//           frees each stage and finally signals the accumulator;
+//   warps 0-3 epilogue: tcgen05.ld of the FP32 accumulator (warp w owns TMEM
+//           lanes 32w..32w+31 = tile rows), scale by s_gA s_gB, round to BF16,
+//           store.
+// Every mbarrier wait is bounded; on a timeout the kernel writes the status word,
+// drains its in-flight copies and MMAs (again bounded), frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+namespace {
+
+template <int BN_>
+struct GemmCfg {
+  static constexpr int BM = 128;
+  static constexpr int BN = BN_;
+  static constexpr int KTILE_BYTES = 128;             // 256 FP4 values per row per stage
+  static constexpr int A_BYTES = BM * KTILE_BYTES;    // 16 KB
+  static constexpr int B_BYTES = BN * KTILE_BYTES;
+  static constexpr int SF_ATOM = 512;                 // 128 rows x 4 scales (64 values of K)
+  static constexpr int SFA_BYTES = 4 * SF_ATOM;       // one row group, 4 K-steps
+  static constexpr int SFB_BYTES = (BN / 128) * 4 * SF_ATOM;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = (220 * 1024) / STAGE_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  // TMEM columns: accumulator [0, BN), A scales 16, B scales BN/8.
+  static constexpr int TMEM_SFA = BN;
+  static constexpr int TMEM_SFB = BN + 16;
+  static constexpr int TMEM_USED = BN + 16 + BN / 8;
+  static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
+  static_assert(BN == 128 || BN == 256, "tile width");
+  static_assert(STAGES >= 2, "pipeline depth");
+};
+
+// Wait with a timeout that ignores the abort flag (teardown after an abort).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(addr, parity)) {
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (status) atomicCAS(status, 0u, static_cast<uint32_t>(kErrWaitDrain));
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat16 a = __float2bfloat16_rn(lo), b = __float2bfloat16_rn(hi);
+  return static_cast<uint32_t>(__bfloat16_as_ushort(a)) | (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb, const float* __restrict__ a_gs,
+                const float* __restrict__ b_gs, uint16_t* __restrict__ C, int M, int N, int K, int64_t ldc,
+                uint32_t* __restrict__ status) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * Cfg::A_BYTES;
+  uint8_t* sSFA = sB + STAGES * Cfg::B_BYTES;
+  uint8_t* sSFB = sSFA + STAGES * Cfg::SFA_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * Cfg::SFB_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile_n = blockIdx.x, tile_m = blockIdx.y;
+  const int k_atoms = (K + 63) / 64;  // 64-value K steps = scale atoms per 128-row group
+  const int k_tiles = (k_atoms + 3) / 4;
+  const int n_groups_b = (N + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_mbarrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int issued_last[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
+      int valid_b_groups = 0;
+      for (int g = 0; g < BN / 128; ++g)
+        if (tile_n * (BN / 128) + g < n_groups_b) ++valid_b_groups;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        const int s = kt % STAGES;
+        const uint32_t ph = static_cast<uint32_t>(kt / STAGES) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status, kErrWaitEmpty)) break;
+        const int ka0 = kt * 4;
+        const int na = min(4, k_atoms - ka0);
+        const uint32_t sf_bytes = static_cast<uint32_t>(na) * Cfg::SF_ATOM;
+        mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + sf_bytes * (1 + valid_b_groups));
+        tma_load_2d(sA + s * Cfg::A_BYTES, &tmap_a, &full[s], kt * Cfg::KTILE_BYTES, tile_m * Cfg::BM);
+        tma_load_2d(sB + s * Cfg::B_BYTES, &tmap_b, &full[s], kt * Cfg::KTILE_BYTES, tile_n * BN);
+        bulk_load(sSFA + s * Cfg::SFA_BYTES, sfa + (static_cast<size_t>(tile_m) * k_atoms + ka0) * Cfg::SF_ATOM,
+                  sf_bytes, &full[s]);
+        for (int g = 0; g < valid_b_groups; ++g)
+          bulk_load(sSFB + s * Cfg::SFB_BYTES + g * 4 * Cfg::SF_ATOM,
+                    sfb + (static_cast<size_t>(tile_n * (BN / 128) + g) * k_atoms + ka0) * Cfg::SF_ATOM, sf_bytes,
+                    &full[s]);
+        issued_last[s] = kt;
+      }
+      if (*abort_flag) {
+        // Let every copy this thread started land before the CTA exits.
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_last[s] >= 0)
+            mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_last[s] / STAGES) & 1u, status);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      const uint32_t idesc = idesc_mxf4nvf4(Cfg::BM, BN);
+      const uint32_t t_acc = tmem_base;
+      const uint32_t t_sfa = tmem_base + Cfg::TMEM_SFA;
+      const uint32_t t_sfb = tmem_base + Cfg::TMEM_SFB;
+      bool ok = true;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        const int s = kt % STAGES;
+        const uint32_t ph = static_cast<uint32_t>(kt / STAGES) & 1u;
+        if (!mbar_wait(&full[s], ph, abort_flag, status, kErrWaitFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int na = min(4, k_atoms - kt * 4);
+        const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
+        const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
+        const uint32_t sfa_base = smem_u32(sSFA + s * Cfg::SFA_BYTES);
+        const uint32_t sfb_base = smem_u32(sSFB + s * Cfg::SFB_BYTES);
+        for (int j = 0; j < na; ++j) {
+          tc_cp_sf(t_sfa + 4 * j, sdesc_sf_tile(sfa_base + j * Cfg::SF_ATOM));
+#pragma unroll
+          for (int g = 0; g < BN / 128; ++g)
+            tc_cp_sf(t_sfb + (BN / 32) * j + 4 * g, sdesc_sf_tile(sfb_base + (g * 4 + j) * Cfg::SF_ATOM));
+        }
+        for (int j = 0; j < na; ++j) {
+          mma_mxf4nvf4(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
+                       t_sfa + 4 * j, t_sfb + (BN / 32) * j, (kt | j) != 0 ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+      }
+      if (ok) {
+        tc_commit(acc_full);
+      } else {
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0u, status);
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 0-3) ----------------
+    if (mbar_wait(acc_full, 0u, abort_flag, status, kErrWaitAccFull)) {
+      tc_fence_after();
+      const float alpha = __fmul_rn(*a_gs, *b_gs);
+      const int row = tile_m * Cfg::BM + warp * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_row + c0, v);
+        tmem_ld_wait();
+        const int col0 = tile_n * BN + c0;
+        if (row < M && col0 < N) {
+          uint32_t p[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            p[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[2 * i]), alpha),
+                               __fmul_rn(__uint_as_float(v[2 * i + 1]), alpha));
+          uint16_t* dst = C + static_cast<int64_t>(row) * ldc + col0;
+          if (col0 + 32 <= N) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          } else {
+            for (int i = 0; i < 32 && col0 + i < N; ++i)
+              dst[i] = static_cast<uint16_t>((i & 1) ? (p[i >> 1] >> 16) : (p[i >> 1] & 0xFFFFu));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// Row-major rows x (K/2) bytes of packed codes, box = box_rows x 128 bytes, 128-byte swizzle.
+bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* a_sf, const uint8_t* b_sf,
+                        const float* a_gs, const float* b_gs, int64_t M, int64_t N, int64_t K, uint16_t* c,
+                        int64_t ldc, uint32_t* status, cudaStream_t stream) {
+  using Cfg = GemmCfg<BN>;
+  static std::once_flag once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(once[dev & 63], [&] {
+    attr_err = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const dim3 grid(static_cast<unsigned>((N + BN - 1) / BN), static_cast<unsigned>((M + Cfg::BM - 1) / Cfg::BM));
+  gemm_kernel<BN><<<grid, 192, Cfg::SMEM_BYTES, stream>>>(ta, tb, a_sf, b_sf, a_gs, b_gs, c, static_cast<int>(M),
+                                                         static_cast<int>(N), static_cast<int>(K), ldc, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
+                        const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
+                        uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream) {
+  const int bn = N > 128 ? 256 : 128;
+  CUtensorMap ta, tb;
+  if (!encode_codes_map(&ta, a_codes, M, K, 128) || !encode_codes_map(&tb, b_codes, N, K, bn))
+    return cudaErrorInvalidValue;
+  if (bn == 256) return launch_tile<256>(ta, tb, a_sf, b_sf, a_gs, b_gs, M, N, K, c, ldc, status, stream);
+  return launch_tile<128>(ta, tb, a_sf, b_sf, a_gs, b_gs, M, N, K, c, ldc, status, stream);
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,31 @@
+// internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+// Quantizer launchers (quantize.cu).  All pointers are device pointers that the
+// API layer has already validated.
+cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax_bits,
+                        cudaStream_t stream);
+cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int mode,
+                            bool swizzled, const float* gs_in, const uint32_t* amax_bits, uint8_t* codes,
+                            uint8_t* scales, float* gs_out, float* block_err, cudaStream_t stream);
+cudaError_t launch_sf_pad_zero(uint8_t* scales, int64_t rows, int64_t nblk, cudaStream_t stream);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, bool swizzled, const float* gs,
+                              int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out, cudaStream_t stream);
+
+// GEMM launcher (gemm_sm100.cu).  Returns cudaErrorInvalidValue when a tensor
+// map cannot be encoded.
+cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
+                        const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
+                        uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream);
+
+// Number of kernel launches the last call of each entry point enqueued (for
+// the benchmark's launch count); host-side bookkeeping only.
+extern thread_local int g_last_launches;
+
+}  // namespace nvfp4

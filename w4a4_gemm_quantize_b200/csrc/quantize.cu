@@ -1,0 +1,345 @@
+// quantize.cu -- NVFP4 block quantization and reconstruction kernels for sm_100a.
+//
+// Method (web page "Tu pipeline NVFP4: meter 62 GB de modelo en 24 GB de laptop",
+// section 2 "Qué es realmente NVFP4"):
+//  * box "Fundamento matemático: bitfield E2M1 y cuantización jerárquica": each
+//    value becomes q = argmin over the E2M1 grid of |x / (s_b s_g) - q|, with s_b an
+//    E4M3 scale per 16 consecutive values and s_g one FP32 scale per tensor;
+//    reconstruction W^ = q s_b s_g;
+//  * box "Derivación del objetivo de optimización MSE vs Absmax": absmax scale
+//    s = max|x| / 6, or the MSE scale that minimises sum_k (x_k - s s_g Q(x_k/(s s_g)))^2
+//    over candidates below the absmax scale (the search of section 8 "Para
+//    practicar" of "NVFP4 en difusión: la misma cuantización, un motor
+//    completamente distinto", with 8 factors 0.3, 0.4, ..., 1.0).
+//
+// Arithmetic, in this order and all binary32 round-to-nearest-even:
+//   s_g = amax_t / 2688 (1 for an all-zero tensor); d6 = 6 s_g; v_b = amax_b / d6;
+//   per candidate f: u = f v_b, s_b = E4M3_sat(u), eff = dec(s_b) s_g, r = 1/eff,
+//   y_k = |x_k| r, mag_k = E2M1_sat(y_k) (RNE), code_k = sign(x_k) | mag_k;
+//   block error e = fma(d_k, d_k, e) over k with d_k = fma(-|q_k|, eff, |x_k|);
+//   candidates walked from f = 1 down, kept on a strict improvement.
+//
+// Kernels are HBM-bound streaming kernels (absmax) or ALU-bound (MSE): one
+// thread per 16-value block, 2 x 128-bit loads per thread, packed 8-byte code
+// stores; hardware cvt for E4M3 and E2M1 rounding.
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// max over the eight BF16 magnitudes of a 16-byte vector, as 16-bit patterns in both halves
+__device__ __forceinline__ uint32_t vmax_mag(uint32_t m, uint4 v) {
+  m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+  m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+  m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+  m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+  return m;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
+
+// Global amax: the largest |x| as the 15-bit magnitude pattern of a BF16 value
+// (for non-negative BF16 values the integer order of the bit patterns is the
+// numeric order).  One atomicMax per CTA into a zero-initialised word.
+__global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                        int64_t cols, int64_t ld,
+                                                        uint32_t* __restrict__ amax_bits) {
+  uint32_t m = 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (ld == cols) {
+    const int64_t nvec = rows * cols / 8;
+    const uint4* v = reinterpret_cast<const uint4*>(x);
+    int64_t i = tid;
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+      uint4 a = ld_nc_v4(v + i), b = ld_nc_v4(v + i + stride), c = ld_nc_v4(v + i + 2 * stride),
+            d = ld_nc_v4(v + i + 3 * stride);
+      m = vmax_mag(m, a);
+      m = vmax_mag(m, b);
+      m = vmax_mag(m, c);
+      m = vmax_mag(m, d);
+    }
+    for (; i < nvec; i += stride) m = vmax_mag(m, ld_nc_v4(v + i));
+  } else {
+    const int64_t vpr = cols / 8;
+    const int64_t nvec = rows * vpr;
+    for (int64_t i = tid; i < nvec; i += stride) {
+      const int64_t r = i / vpr, c = i - r * vpr;
+      m = vmax_mag(m, ld_nc_v4(x + r * ld + c * 8));
+    }
+  }
+  m = max(m & 0xFFFFu, m >> 16);
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t warp_max[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < kThreads / 32 ? warp_max[threadIdx.x] : 0u;
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (threadIdx.x == 0 && m != 0) atomicMax(amax_bits, m);
+  }
+}
+
+// Magnitude codes of 16 values for effective scale eff (eff == 0: all zero).
+__device__ __forceinline__ void encode_mags(const float (&ax)[16], float eff, uint32_t& c0, uint32_t& c1) {
+  if (eff == 0.0f) {
+    c0 = c1 = 0u;
+    return;
+  }
+  const float r = __frcp_rn(eff);
+  float y[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) y[k] = __fmul_rn(ax[k], r);
+  if (isinf(r)) {
+    // 1/eff overflowed: a zero input gives 0 * inf = NaN; it encodes as 0.
+#pragma unroll
+    for (int k = 0; k < 16; ++k) y[k] = fmaxf(y[k], 0.0f);
+  }
+  c0 = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+  c1 = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+}
+
+// Squared reconstruction error of the block, accumulated in element order.
+__device__ __forceinline__ float block_sse(const float (&ax)[16], uint32_t c0, uint32_t c1, float eff) {
+  float e = 0.0f;
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const uint32_t word = w ? c1 : c0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t h2 = e2m1x2_to_half2(word, k);
+      const float q_lo = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFFu)));
+      const float q_hi = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 >> 16)));
+      const float d0 = __fmaf_rn(-q_lo, eff, ax[8 * w + 2 * k]);
+      e = __fmaf_rn(d0, d0, e);
+      const float d1 = __fmaf_rn(-q_hi, eff, ax[8 * w + 2 * k + 1]);
+      e = __fmaf_rn(d1, d1, e);
+    }
+  }
+  return e;
+}
+
+// Sign bits of eight BF16 values (words w0..w3, two values each) moved to bit 3
+// of their nibble in a packed code word.
+__device__ __forceinline__ uint32_t sign_nibbles(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  return ((w0 >> 12) & 0x8u) | ((w0 >> 24) & 0x80u) | ((w1 >> 4) & 0x800u) | ((w1 >> 16) & 0x8000u) |
+         ((w2 << 4) & 0x80000u) | ((w2 >> 8) & 0x800000u) | ((w3 << 12) & 0x8000000u) |
+         (w3 & 0x80000000u);
+}
+
+__device__ __forceinline__ int64_t swizzled_offset(int64_t r, int64_t c, int64_t atoms_per_group) {
+  return ((r >> 7) * atoms_per_group + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+__device__ __forceinline__ float global_scale(const float* gs_in, const uint32_t* amax_bits) {
+  if (gs_in) return *gs_in;
+  const float amax = bf16_bits_to_float(*amax_bits);
+  return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
+}
+
+template <int MODE, bool SWZ>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, const float* __restrict__ gs_in,
+    const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+    float* __restrict__ gs_out, float* __restrict__ block_err) {
+  const int64_t nblk = cols / 16;
+  const int64_t total = rows * nblk;
+  const int64_t atoms_per_group = (nblk + 3) / 4;
+  const float sg = global_scale(gs_in, amax_bits);
+  if (gs_out && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = sg;
+  const float d6 = __fmul_rn(6.0f, sg);
+
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total; b += stride) {
+    const int64_t r = b / nblk, cb = b - r * nblk;
+    const uint16_t* src = x + r * ld + cb * 16;
+    const uint4 lo = ld_nc_v4(src), hi = ld_nc_v4(src + 8);
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    float ax[16];
+    uint32_t mb = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      ax[2 * i] = bf16_bits_to_float(w[i] & 0x7FFFu);
+      ax[2 * i + 1] = bf16_bits_to_float((w[i] >> 16) & 0x7FFFu);
+      mb = __vmaxu2(mb, w[i] & 0x7FFF7FFFu);
+    }
+    const float amax_b = bf16_bits_to_float(max(mb & 0xFFFFu, mb >> 16));
+    const float vb = __fdiv_rn(amax_b, d6);
+
+    // candidate f = 1: the absmax scale
+    uint32_t best_s = cvt_e4m3_satfinite(vb);
+    float best_eff = __fmul_rn(e4m3_to_float(best_s), sg);
+    uint32_t best_c0, best_c1;
+    encode_mags(ax, best_eff, best_c0, best_c1);
+    float best_e = 0.0f;
+    if (MODE == 1 || block_err) best_e = block_sse(ax, best_c0, best_c1, best_eff);
+
+    if (MODE == 1) {
+      const float factors[7] = {0.9f, 0.8f, 0.7f, 0.6f, 0.5f, 0.4f, 0.3f};
+      uint32_t prev_s = best_s;
+#pragma unroll
+      for (int i = 0; i < 7; ++i) {
+        const uint32_t s = cvt_e4m3_satfinite(__fmul_rn(factors[i], vb));
+        if (s == prev_s) continue;  // same scale, same error: never a strict improvement
+        prev_s = s;
+        const float eff = __fmul_rn(e4m3_to_float(s), sg);
+        uint32_t c0, c1;
+        encode_mags(ax, eff, c0, c1);
+        const float e = block_sse(ax, c0, c1, eff);
+        if (e < best_e) {
+          best_e = e;
+          best_s = s;
+          best_c0 = c0;
+          best_c1 = c1;
+        }
+      }
+    }
+
+    best_c0 |= sign_nibbles(w[0], w[1], w[2], w[3]);
+    best_c1 |= sign_nibbles(w[4], w[5], w[6], w[7]);
+    *reinterpret_cast<uint2*>(codes + r * (cols / 2) + cb * 8) = make_uint2(best_c0, best_c1);
+    if (SWZ)
+      scales[swizzled_offset(r, cb, atoms_per_group)] = static_cast<uint8_t>(best_s);
+    else
+      scales[b] = static_cast<uint8_t>(best_s);
+    if (block_err) block_err[b] = best_e;
+  }
+}
+
+// Zero the padding of a swizzled scale buffer: rows [rows, Rp) and block columns
+// [nblk, Cp) of rows [0, rows).
+__global__ void sf_pad_zero_kernel(uint8_t* __restrict__ scales, int64_t rows, int64_t nblk) {
+  const int64_t rp = (rows + 127) / 128 * 128;
+  const int64_t cp = (nblk + 3) / 4 * 4;
+  const int64_t atoms_per_group = cp / 4;
+  const int64_t n_row_pad = (rp - rows) * cp;
+  const int64_t n_col_pad = rows * (cp - nblk);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_row_pad + n_col_pad;
+       i += stride) {
+    int64_t r, c;
+    if (i < n_row_pad) {
+      r = rows + i / cp;
+      c = i % cp;
+    } else {
+      const int64_t j = i - n_row_pad;
+      const int64_t w = cp - nblk;
+      r = j / w;
+      c = nblk + j % w;
+    }
+    scales[swizzled_offset(r, c, atoms_per_group)] = 0;
+  }
+}
+
+template <bool SWZ>
+__global__ void __launch_bounds__(kThreads) dequantize_kernel(const uint8_t* __restrict__ codes,
+                                                              const uint8_t* __restrict__ scales,
+                                                              const float* __restrict__ gs, int64_t rows,
+                                                              int64_t cols, uint16_t* __restrict__ out,
+                                                              int64_t ld_out) {
+  const int64_t nblk = cols / 16;
+  const int64_t total = rows * nblk;
+  const int64_t atoms_per_group = (nblk + 3) / 4;
+  const float sg = *gs;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total; b += stride) {
+    const int64_t r = b / nblk, cb = b - r * nblk;
+    const uint2 cw = *reinterpret_cast<const uint2*>(codes + r * (cols / 2) + cb * 8);
+    const uint32_t s = SWZ ? scales[swizzled_offset(r, cb, atoms_per_group)] : scales[b];
+    const float eff = __fmul_rn(e4m3_to_float(s), sg);
+    uint32_t o[8];
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const uint32_t word = w ? cw.y : cw.x;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t h2 = e2m1x2_to_half2(word, k);
+        const float q_lo = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFFu)));
+        const float q_hi = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 >> 16)));
+        const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(q_lo, eff));
+        const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(q_hi, eff));
+        o[4 * w + k] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+                       (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + r * ld_out + cb * 16);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+int grid_for(int64_t work, int threads) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t need = (work + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(sms) * 16;  // grid-stride beyond 16 CTAs per SM
+  return static_cast<int>(need < 1 ? 1 : (need < cap ? need : cap));
+}
+
+}  // namespace
+
+cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax_bits,
+                        cudaStream_t stream) {
+  const int64_t vecs = rows * cols / 8;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t blocks = (vecs + kThreads * 4 - 1) / (kThreads * 4);
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  amax_kernel<<<static_cast<int>(blocks), kThreads, 0, stream>>>(x, rows, cols, ld, amax_bits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int mode,
+                            bool swizzled, const float* gs_in, const uint32_t* amax_bits, uint8_t* codes,
+                            uint8_t* scales, float* gs_out, float* block_err, cudaStream_t stream) {
+  const int64_t blocks16 = rows * (cols / 16);
+  const int grid = grid_for(blocks16, kThreads);
+#define NVFP4_Q(MODE, SWZ)                                                                                 \
+  quantize_kernel<MODE, SWZ><<<grid, kThreads, 0, stream>>>(x, rows, cols, ld, gs_in, amax_bits, codes, \
+                                                            scales, gs_out, block_err)
+  if (mode == 1) {
+    if (swizzled) NVFP4_Q(1, true); else NVFP4_Q(1, false);
+  } else {
+    if (swizzled) NVFP4_Q(0, true); else NVFP4_Q(0, false);
+  }
+#undef NVFP4_Q
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sf_pad_zero(uint8_t* scales, int64_t rows, int64_t nblk, cudaStream_t stream) {
+  const int64_t rp = (rows + 127) / 128 * 128, cp = (nblk + 3) / 4 * 4;
+  const int64_t pads = (rp - rows) * cp + rows * (cp - nblk);
+  if (pads == 0) return cudaSuccess;
+  sf_pad_zero_kernel<<<grid_for(pads, kThreads), kThreads, 0, stream>>>(scales, rows, nblk);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, bool swizzled, const float* gs,
+                              int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out, cudaStream_t stream) {
+  const int grid = grid_for(rows * (cols / 16), kThreads);
+  if (swizzled)
+    dequantize_kernel<true><<<grid, kThreads, 0, stream>>>(codes, scales, gs, rows, cols, out, ld_out);
+  else
+    dequantize_kernel<false><<<grid, kThreads, 0, stream>>>(codes, scales, gs, rows, cols, out, ld_out);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4
