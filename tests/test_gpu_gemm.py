@@ -87,7 +87,7 @@ def test_zero_and_sign_cases(cuda_device):
 def test_integer_grid_special_case(cuda_device):
     """All block scales 1 and s_g = 1: C is an exact integer matmul / 4."""
     r = np.random.default_rng(12)
-    M, N, K = 130, 260, 320
+    M, N, K = 130, 264, 320
     ca = r.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
     cb = r.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
     sa = np.full((M, K // 16), 0x38, np.uint8)
