@@ -145,6 +145,28 @@ nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const f
  * next nvfp4_gemm that uses it. */
 nvfp4_status nvfp4_read_device_error(const void *workspace, void *stream, uint32_t *word);
 
+/* nvfp4_quantize for callers that cannot allocate device memory: a framework or
+ * server plugin that owns no allocator and gets no workspace from its host, or a
+ * latency-critical loop where cudaMalloc would synchronize the device.  Same
+ * arguments and results as nvfp4_quantize, minus the workspace: it uses a
+ * 256-byte scratch block compiled into the library (one per GPU, held until the
+ * process exits).  The pages have no counterpart; this is an interface of this
+ * library only.
+ *  - It allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ *  - The first call on a device, with that device current, looks up the scratch
+ *    block's device address (cudaGetSymbolAddress); make that first call before
+ *    any stream capture.
+ *  - Every call shares the one scratch block per device and clears what it needs
+ *    zeroed before use; calls whose work overlaps on the GPU (other streams, or
+ *    other host threads) race on it -- serialize them.
+ *  - Returns NVFP4_ERR_WORKSPACE if the quantizer would need more scratch than
+ *    the 256 bytes (nvfp4_quantize_workspace_bytes(rows, cols) > 256); otherwise
+ *    the errors of nvfp4_quantize. */
+nvfp4_status nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                                    nvfp4_scale_mode mode, nvfp4_sf_layout layout,
+                                    const float *global_scale_in, uint8_t *codes, uint8_t *scales,
+                                    float *global_scale_out, float *block_err, void *stream);
+
 /* Number of kernels the most recent nvfp4_quantize / nvfp4_dequantize /
  * nvfp4_gemm call on the calling host thread enqueued (library bookkeeping for
  * launch counting; no counterpart on the pages). */

@@ -51,6 +51,7 @@ SIGNATURES = {
     "nvfp4_gemm": ([_P, _P, _P, _I64, _P, _P, _P, _I64, _I64, _P, _I64, _P, _SZ, _P], _I),
     "nvfp4_read_device_error": ([_P, _P, ctypes.POINTER(ctypes.c_uint32)], _I),
     "nvfp4_last_launch_count": ([], _I),
+    "nvfp4_quantize_noalloc": ([_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P, _P, _P], _I),
 }
 
 
@@ -143,6 +144,33 @@ def nvfp4_quantize(x: torch.Tensor, mode="absmax", layout="swizzled", global_sca
                             _ptr(out.scales), _ptr(out.global_scale), _ptr(out.block_err), _ptr(workspace),
                             ws_bytes, _stream(stream))
     _check(st, "nvfp4_quantize")
+    return out
+
+
+def nvfp4_quantize_noalloc(x: torch.Tensor, mode="absmax", layout="swizzled",
+                           global_scale: Optional[torch.Tensor] = None, block_err: bool = False,
+                           out: Optional[NVFP4Tensor] = None, stream=None) -> NVFP4Tensor:
+    """nvfp4_quantize without a workspace, for callers that cannot allocate device
+    memory: the library's own 256-byte scratch block per GPU is used instead.
+    Calls that overlap on the GPU share that block and race; serialize them."""
+    lib = load_library()
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D row-major bfloat16 CUDA tensor")
+    rows, cols = x.shape
+    lay = _LAYOUTS[layout]
+    if out is None:
+        dev = x.device
+        codes = torch.empty(lib.nvfp4_codes_bytes(rows, cols), dtype=torch.uint8, device=dev).view(rows, cols // 2)
+        scales = torch.empty(lib.nvfp4_scales_bytes(rows, cols, lay), dtype=torch.uint8, device=dev)
+        if lay == SF_LINEAR:
+            scales = scales.view(rows, cols // 16)
+        gs = torch.empty(1, dtype=torch.float32, device=dev)
+        err = torch.empty((rows, cols // 16), dtype=torch.float32, device=dev) if block_err else None
+        out = NVFP4Tensor(codes, scales, gs, rows, cols, lay, err)
+    st = lib.nvfp4_quantize_noalloc(_ptr(x), rows, cols, x.stride(0), _MODES[mode], lay, _ptr(global_scale),
+                                    _ptr(out.codes), _ptr(out.scales), _ptr(out.global_scale),
+                                    _ptr(out.block_err), _stream(stream))
+    _check(st, "nvfp4_quantize_noalloc")
     return out
 
 
