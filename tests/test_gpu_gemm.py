@@ -74,6 +74,15 @@ def test_ragged_shapes_full_compare(cuda_device, M, N, K):
     run_full(oracle_operand(xa), oracle_operand(xb, oracle.SCALE_MSE), M, N, K)
 
 
+@pytest.mark.parametrize("M,N,K", [(1280, 4096, 128), (2176, 2560, 96)])
+def test_more_tiles_than_sms_full_compare(cuda_device, M, N, K):
+    """More output tiles than SMs, so each persistent CTA walks several tiles (and the
+    grouped tile order ends on a partial group of row tiles)."""
+    xa = workloads.activation(M, K, seed=M + 1, n_outlier_channels=2)
+    xb = workloads.gaussian_weight(N, K, 0.02, seed=N + 1)
+    run_full(oracle_operand(xa), oracle_operand(xb, oracle.SCALE_MSE), M, N, K)
+
+
 def test_zero_and_sign_cases(cuda_device):
     M, N, K = 64, 256, 256
     z = workloads.to_bf16(np.zeros((M, K), np.float32))

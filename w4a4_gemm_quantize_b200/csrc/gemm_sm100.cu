@@ -6,18 +6,21 @@
 // vLLM: torch._scaled_mm a mano" -- the per-16 E4M3 scales travel as separate
 // tensors and are applied per block inside the kernel; the result is BF16.
 //
-// Design (one CTA per 128 x BN output tile, 6 warps):
-//   warp 4  TMA producer: per K-tile of 256 values, a 128 x 128-byte A tile and a
+// Design: a persistent kernel, one CTA per SM, each CTA walking 128 x BN output
+// tiles in a grouped order (GROUP_M row-tiles at a time, so the CTAs running at
+// the same moment share A and B tiles through L2).  Ten warps:
+//   warp 8  TMA producer: per K-tile of 256 values, a 128 x 128-byte A tile and a
 //           BN x 128-byte B tile (tensor maps, 128-byte swizzle) plus the scale
 //           tiles (plain bulk copies of the 512-byte 128x4 atoms), into a
-//           STAGES-deep shared-memory ring guarded by full/empty mbarriers;
-//   warp 5  allocates TMEM and issues, from one thread, tcgen05.cp of the scale
+//           STAGES-deep shared-memory ring guarded by full/empty mbarriers; the
+//           ring keeps flowing across tile boundaries;
+//   warp 9  allocates TMEM and issues, from one thread, tcgen05.cp of the scale
 //           atoms into TMEM and tcgen05.mma.kind::mxf4nvf4.block_scale.block16
-//           (128 x BN x 64 per instruction) accumulating in TMEM; tcgen05.commit
-//           frees each stage and finally signals the accumulator;
-//   warps 0-3 epilogue: tcgen05.ld of the FP32 accumulator (warp w owns TMEM
-//           lanes 32w..32w+31 = tile rows), scale by s_gA s_gB, round to BF16,
-//           store.
+//           (128 x BN x 64 per instruction) into the TMEM accumulator;
+//           tcgen05.commit frees each stage and signals the finished tile;
+//   warps 0-7 epilogue: warp w reads TMEM lanes 32(w%4).. (tile rows) and half of
+//           the columns, converts to BF16 in registers, releases the accumulator
+//           (so the next tile's MMAs start) and then stores its rows.
 // Every mbarrier wait is bounded; on a timeout the kernel writes the status word,
 // drains its in-flight copies and MMAs (again bounded), frees TMEM and returns.
 #include <cuda.h>
@@ -46,6 +49,11 @@ struct GemmCfg {
   static constexpr int STAGES = (220 * 1024) / STAGE_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int PRODUCER_WARP = EPI_WARPS;
+  static constexpr int MMA_WARP = EPI_WARPS + 1;
+  static constexpr int THREADS = (EPI_WARPS + 2) * 32;
+  static constexpr int GROUP_M = 8;
   // TMEM columns: accumulator [0, BN), A scales 16, B scales BN/8.
   static constexpr int TMEM_SFA = BN;
   static constexpr int TMEM_SFB = BN + 16;
@@ -73,8 +81,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(a)) | (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
 }
 
+// Tile t -> (row tile, column tile): groups of GROUP_M row tiles, column-major
+// inside a group, so that consecutive tiles reuse the same few A and B tiles.
+template <int GROUP_M>
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& tm, int& tn) {
+  const int per_group = GROUP_M * num_n;
+  const int g = t / per_group;
+  const int first_m = g * GROUP_M;
+  const int gm = min(GROUP_M, num_m - first_m);
+  const int local = t - g * per_group;
+  tm = first_m + local % gm;
+  tn = local / gm;
+}
+
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                 const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb, const float* __restrict__ a_gs,
                 const float* __restrict__ b_gs, uint16_t* __restrict__ C, int M, int N, int K, int64_t ldc,
@@ -90,15 +111,18 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * Cfg::SFB_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
-  uint64_t* drain = acc_full + 1;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile_n = blockIdx.x, tile_m = blockIdx.y;
   const int k_atoms = (K + 63) / 64;  // 64-value K steps = scale atoms per 128-row group
   const int k_tiles = (k_atoms + 3) / 4;
   const int n_groups_b = (N + 127) / 128;
+  const int num_m = (M + Cfg::BM - 1) / Cfg::BM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -106,15 +130,16 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, Cfg::EPI_WARPS);
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_mbarrier_init();
   }
-  if (warp == 5) {
+  if (warp == Cfg::MMA_WARP) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == Cfg::PRODUCER_WARP && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
   }
@@ -123,32 +148,41 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == Cfg::PRODUCER_WARP) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       int issued_last[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
-      int valid_b_groups = 0;
-      for (int g = 0; g < BN / 128; ++g)
-        if (tile_n * (BN / 128) + g < n_groups_b) ++valid_b_groups;
-      for (int kt = 0; kt < k_tiles; ++kt) {
-        const int s = kt % STAGES;
-        const uint32_t ph = static_cast<uint32_t>(kt / STAGES) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status, kErrWaitEmpty)) break;
-        const int ka0 = kt * 4;
-        const int na = min(4, k_atoms - ka0);
-        const uint32_t sf_bytes = static_cast<uint32_t>(na) * Cfg::SF_ATOM;
-        mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + sf_bytes * (1 + valid_b_groups));
-        tma_load_2d(sA + s * Cfg::A_BYTES, &tmap_a, &full[s], kt * Cfg::KTILE_BYTES, tile_m * Cfg::BM);
-        tma_load_2d(sB + s * Cfg::B_BYTES, &tmap_b, &full[s], kt * Cfg::KTILE_BYTES, tile_n * BN);
-        bulk_load(sSFA + s * Cfg::SFA_BYTES, sfa + (static_cast<size_t>(tile_m) * k_atoms + ka0) * Cfg::SF_ATOM,
-                  sf_bytes, &full[s]);
-        for (int g = 0; g < valid_b_groups; ++g)
-          bulk_load(sSFB + s * Cfg::SFB_BYTES + g * 4 * Cfg::SF_ATOM,
-                    sfb + (static_cast<size_t>(tile_n * (BN / 128) + g) * k_atoms + ka0) * Cfg::SF_ATOM, sf_bytes,
-                    &full[s]);
-        issued_last[s] = kt;
+      int kc = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int tm, tn;
+        tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
+        int valid_b_groups = 0;
+        for (int g = 0; g < BN / 128; ++g)
+          if (tn * (BN / 128) + g < n_groups_b) ++valid_b_groups;
+        for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+          const int s = kc % STAGES;
+          const uint32_t ph = static_cast<uint32_t>(kc / STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          const int ka0 = kt * 4;
+          const int na = min(4, k_atoms - ka0);
+          const uint32_t sf_bytes = static_cast<uint32_t>(na) * Cfg::SF_ATOM;
+          mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + sf_bytes * (1 + valid_b_groups));
+          tma_load_2d(sA + s * Cfg::A_BYTES, &tmap_a, &full[s], kt * Cfg::KTILE_BYTES, tm * Cfg::BM);
+          tma_load_2d(sB + s * Cfg::B_BYTES, &tmap_b, &full[s], kt * Cfg::KTILE_BYTES, tn * BN);
+          bulk_load(sSFA + s * Cfg::SFA_BYTES, sfa + (static_cast<size_t>(tm) * k_atoms + ka0) * Cfg::SF_ATOM,
+                    sf_bytes, &full[s]);
+          for (int g = 0; g < valid_b_groups; ++g)
+            bulk_load(sSFB + s * Cfg::SFB_BYTES + g * 4 * Cfg::SF_ATOM,
+                      sfb + (static_cast<size_t>(tn * (BN / 128) + g) * k_atoms + ka0) * Cfg::SF_ATOM, sf_bytes,
+                      &full[s]);
+          issued_last[s] = kc;
+        }
       }
       if (*abort_flag) {
         // Let every copy this thread started land before the CTA exits.
@@ -157,7 +191,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_last[s] / STAGES) & 1u, status);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == Cfg::MMA_WARP) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
       const uint32_t idesc = idesc_mxf4nvf4(Cfg::BM, BN);
@@ -165,66 +199,86 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t t_sfa = tmem_base + Cfg::TMEM_SFA;
       const uint32_t t_sfb = tmem_base + Cfg::TMEM_SFB;
       bool ok = true;
-      for (int kt = 0; kt < k_tiles; ++kt) {
-        const int s = kt % STAGES;
-        const uint32_t ph = static_cast<uint32_t>(kt / STAGES) & 1u;
-        if (!mbar_wait(&full[s], ph, abort_flag, status, kErrWaitFull)) {
+      int kc = 0, it = 0;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++it) {
+        // the epilogue must have drained the previous tile's accumulator
+        if (!mbar_wait(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, status, kErrWaitAccEmpty)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int na = min(4, k_atoms - kt * 4);
-        const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
-        const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
-        const uint32_t sfa_base = smem_u32(sSFA + s * Cfg::SFA_BYTES);
-        const uint32_t sfb_base = smem_u32(sSFB + s * Cfg::SFB_BYTES);
-        for (int j = 0; j < na; ++j) {
-          tc_cp_sf(t_sfa + 4 * j, sdesc_sf_tile(sfa_base + j * Cfg::SF_ATOM));
+        for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+          const int s = kc % STAGES;
+          const uint32_t ph = static_cast<uint32_t>(kc / STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag, status, kErrWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int na = min(4, k_atoms - kt * 4);
+          const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
+          const uint32_t sfa_base = smem_u32(sSFA + s * Cfg::SFA_BYTES);
+          const uint32_t sfb_base = smem_u32(sSFB + s * Cfg::SFB_BYTES);
+          for (int j = 0; j < na; ++j) {
+            tc_cp_sf(t_sfa + 4 * j, sdesc_sf_tile(sfa_base + j * Cfg::SF_ATOM));
 #pragma unroll
-          for (int g = 0; g < BN / 128; ++g)
-            tc_cp_sf(t_sfb + (BN / 32) * j + 4 * g, sdesc_sf_tile(sfb_base + (g * 4 + j) * Cfg::SF_ATOM));
+            for (int g = 0; g < BN / 128; ++g)
+              tc_cp_sf(t_sfb + (BN / 32) * j + 4 * g, sdesc_sf_tile(sfb_base + (g * 4 + j) * Cfg::SF_ATOM));
+          }
+          for (int j = 0; j < na; ++j) {
+            mma_mxf4nvf4(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
+                         t_sfa + 4 * j, t_sfb + (BN / 32) * j, (kt | j) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
         }
-        for (int j = 0; j < na; ++j) {
-          mma_mxf4nvf4(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
-                       t_sfa + 4 * j, t_sfb + (BN / 32) * j, (kt | j) != 0 ? 1u : 0u);
-        }
-        tc_commit(&empty[s]);
-      }
-      if (ok) {
+        if (!ok) break;
         tc_commit(acc_full);
-      } else {
+      }
+      if (!ok) {
         tc_commit(drain);
         mbar_wait_drain(drain, 0u, status);
       }
     }
   } else {
-    // ---------------- epilogue (warps 0-3) ----------------
-    if (mbar_wait(acc_full, 0u, abort_flag, status, kErrWaitAccFull)) {
+    // ---------------- epilogue (warps 0-7) ----------------
+    constexpr int HALF = BN / 2;  // columns per epilogue warp
+    const int quarter = warp & 3, half = warp >> 2;
+    const float alpha = __fmul_rn(*a_gs, *b_gs);
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * HALF;
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      int tm, tn;
+      tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
+      if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, kErrWaitAccFull)) break;
       tc_fence_after();
-      const float alpha = __fmul_rn(*a_gs, *b_gs);
-      const int row = tile_m * Cfg::BM + warp * 32 + lane;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      uint32_t p[HALF / 2];
+#pragma unroll
+      for (int c = 0; c < HALF; c += 32) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(t_row + c0, v);
+        tmem_ld_32x32b_x32(t_lane + c, v);
         tmem_ld_wait();
-        const int col0 = tile_n * BN + c0;
-        if (row < M && col0 < N) {
-          uint32_t p[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            p[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[2 * i]), alpha),
-                               __fmul_rn(__uint_as_float(v[2 * i + 1]), alpha));
-          uint16_t* dst = C + static_cast<int64_t>(row) * ldc + col0;
-          if (col0 + 32 <= N) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
+        for (int i = 0; i < 16; ++i)
+          p[c / 2 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[2 * i]), alpha),
+                                     __fmul_rn(__uint_as_float(v[2 * i + 1]), alpha));
+      }
+      // accumulator drained: let the MMA warp start the next tile
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      const int row = tm * Cfg::BM + quarter * 32 + lane;
+      const int col0 = tn * BN + half * HALF;
+      if (row < M && col0 < N) {
+        uint16_t* dst = C + static_cast<int64_t>(row) * ldc + col0;
+        if (col0 + HALF <= N) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-          } else {
-            for (int i = 0; i < 32 && col0 + i < N; ++i)
-              dst[i] = static_cast<uint16_t>((i & 1) ? (p[i >> 1] >> 16) : (p[i >> 1] & 0xFFFFu));
-          }
+          for (int i = 0; i < HALF / 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < HALF; ++i)
+            if (col0 + i < N) dst[i] = static_cast<uint16_t>((i & 1) ? (p[i >> 1] >> 16) : (p[i >> 1] & 0xFFFFu));
         }
       }
     }
@@ -232,7 +286,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == Cfg::MMA_WARP) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
@@ -285,9 +339,13 @@ cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint
     attr_err = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  const dim3 grid(static_cast<unsigned>((N + BN - 1) / BN), static_cast<unsigned>((M + Cfg::BM - 1) / Cfg::BM));
-  gemm_kernel<BN><<<grid, 192, Cfg::SMEM_BYTES, stream>>>(ta, tb, a_sf, b_sf, a_gs, b_gs, c, static_cast<int>(M),
-                                                         static_cast<int>(N), static_cast<int>(K), ldc, status);
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + BN - 1) / BN);
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  gemm_kernel<BN><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, a_sf, b_sf, a_gs, b_gs, c,
+                                                                   static_cast<int>(M), static_cast<int>(N),
+                                                                   static_cast<int>(K), ldc, status);
   return cudaGetLastError();
 }
 
