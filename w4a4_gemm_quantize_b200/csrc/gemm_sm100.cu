@@ -54,13 +54,15 @@ struct GemmCfg {
   static constexpr int MMA_WARP = EPI_WARPS + 1;
   static constexpr int THREADS = (EPI_WARPS + 2) * 32;
   static constexpr int GROUP_M = 8;
-  // TMEM columns: accumulator [0, BN), A scales 16, B scales BN/8.
+  // TMEM columns: accumulator [0, BN), then two scale regions (A 16 + B BN/8 each).
   static constexpr int TMEM_SFA = BN;
   static constexpr int TMEM_SFB = BN + 16;
-  static constexpr int TMEM_USED = BN + 16 + BN / 8;
+  static constexpr int TMEM_SF_STRIDE = 16 + BN / 8;
+  static constexpr int TMEM_USED = BN + 2 * TMEM_SF_STRIDE;
   static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
   static_assert(BN == 128 || BN == 256, "tile width");
   static_assert(STAGES >= 2, "pipeline depth");
+  static_assert(TMEM_USED <= TMEM_COLS, "TMEM budget");
 };
 
 // Wait with a timeout that ignores the abort flag (teardown after an abort).
@@ -220,15 +222,17 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
           const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
           const uint32_t sfa_base = smem_u32(sSFA + s * Cfg::SFA_BYTES);
           const uint32_t sfb_base = smem_u32(sSFB + s * Cfg::SFB_BYTES);
+          // scale factors go to one of two TMEM regions by K-tile parity, so these
+          // copies need not wait for the previous K-tile's MMAs to finish reading
+          const uint32_t sf_off = (kc & 1) ? Cfg::TMEM_SF_STRIDE : 0u;
           for (int j = 0; j < na; ++j) {
-            tc_cp_sf(t_sfa + 4 * j, sdesc_sf_tile(sfa_base + j * Cfg::SF_ATOM));
+            tc_cp_sf(t_sfa + sf_off + 4 * j, sdesc_sf_tile(sfa_base + j * Cfg::SF_ATOM));
 #pragma unroll
             for (int g = 0; g < BN / 128; ++g)
-              tc_cp_sf(t_sfb + (BN / 32) * j + 4 * g, sdesc_sf_tile(sfb_base + (g * 4 + j) * Cfg::SF_ATOM));
-          }
-          for (int j = 0; j < na; ++j) {
+              tc_cp_sf(t_sfb + sf_off + (BN / 32) * j + 4 * g,
+                       sdesc_sf_tile(sfb_base + (g * 4 + j) * Cfg::SF_ATOM));
             mma_mxf4nvf4(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
-                         t_sfa + 4 * j, t_sfb + (BN / 32) * j, (kt | j) != 0 ? 1u : 0u);
+                         t_sfa + sf_off + 4 * j, t_sfb + sf_off + (BN / 32) * j, (kt | j) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[s]);
         }
@@ -294,6 +298,334 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------------------------
+// CTA-pair kernel: tcgen05 cta_group::2, 256 x 256 output tile per pair of SMs
+// ---------------------------------------------------------------------------------------------
+//
+// The two CTAs of a cluster share one MMA: CTA r holds rows 128r..128r+127 of the
+// tile's A block and rows 128r..128r+127 of its B block in shared memory; the
+// leader (rank 0) issues every tcgen05.mma for the pair and each CTA's TMEM holds
+// its 128 accumulator rows.  Each CTA's producer loads its A/B halves with pair
+// TMA loads that complete on the leader's `full` barrier (the leader expects the
+// pair's bytes); the leader's commits arrive on both CTAs' barriers.
+//
+// Scale factors: each CTA loads its own 128 rows of A scales and all 256 rows of B
+// scales (one K-tile: 4 + 8 atoms of 512 bytes) with single-CTA TMA loads, and
+// "scale warps" copy them from shared memory into the TMEM scale region of that
+// pipeline stage with tcgen05.st: the four warps of a set cover the four 32-lane
+// TMEM sub-partitions and every lane writes the same 16-byte atom line, which is
+// the 4-way replication the block-scaled MMA reads.  This keeps the copy off the
+// tensor pipe (tcgen05.cp of the same bytes, even one copy per MMA, serialises with
+// the MMAs).  Three sets rotate over K-tiles so that one set's barrier round trip
+// overlaps the others' copies.  A stage's region is free again when its
+// shared-memory slot is: the producer reloads stage s only after the MMAs that
+// read it completed, so no separate release barrier is needed.
+//
+// Epilogue: 8 warps (2 per sub-partition) read the accumulator, release it, and
+// write BF16 through 128-byte-swizzled shared-memory boxes with TMA stores.
+
+struct PairCfg {
+  static constexpr int BM = 128;                      // rows of A per CTA (256 per pair)
+  static constexpr int BN = 256;                      // columns of the pair's tile
+  static constexpr int KTILE_BYTES = 128;             // 256 FP4 values per row per stage
+  static constexpr int A_BYTES = BM * KTILE_BYTES;    // 16 KB
+  static constexpr int B_BYTES = 128 * KTILE_BYTES;   // this CTA's half of B: 16 KB
+  static constexpr int SF_ATOM = 512;
+  static constexpr int SFA_BYTES = 4 * SF_ATOM;       // own 128 rows, 4 K-steps
+  static constexpr int SFB_BYTES = 2 * 4 * SF_ATOM;   // all 256 rows, 4 K-steps
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = 5;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int C_BOX_BYTES = 32 * 128;        // 32 rows x 64 BF16 columns
+  static constexpr int C_BYTES = EPI_WARPS * C_BOX_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + C_BYTES + BAR_BYTES;
+  static constexpr int PRODUCER_WARP = EPI_WARPS;     // 8
+  static constexpr int MMA_WARP = EPI_WARPS + 1;      // 9
+  static constexpr int SF_WARP0 = EPI_WARPS + 2;      // 10..
+  static constexpr int SF_SETS = 3;                   // sets of 4 scale warps, rotating over K-tiles
+  static constexpr int THREADS = (EPI_WARPS + 2 + 4 * SF_SETS) * 32;
+  static constexpr int GROUP_M = 8;                   // in 256-row tiles
+  static constexpr int SF_REGIONS = STAGES;           // one TMEM scale region per pipeline stage
+  static constexpr int SF_COLS = 48;                  // A: 16 columns, B: 32 columns per K-tile
+  static constexpr int TMEM_SF = BN;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(BN + SF_REGIONS * SF_COLS <= TMEM_COLS, "TMEM budget");
+};
+
+__global__ void __launch_bounds__(PairCfg::THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                     const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                     const __grid_constant__ CUtensorMap tmap_c, const float* __restrict__ a_gs,
+                     const float* __restrict__ b_gs, int M, int N, int K, uint32_t* __restrict__ status) {
+  using Cfg = PairCfg;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr int R = Cfg::SF_REGIONS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * Cfg::A_BYTES;
+  uint8_t* sSFA = sB + STAGES * Cfg::B_BYTES;
+  uint8_t* sSFB = sSFA + STAGES * Cfg::SFA_BYTES;
+  uint8_t* sC = sSFB + STAGES * Cfg::SFB_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sC + Cfg::C_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* sf_full = empty + STAGES;
+  uint64_t* sf_ready = sf_full + STAGES;
+  uint64_t* acc_full = sf_ready + R;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = static_cast<int>(cluster_id_x());
+  const int npairs = static_cast<int>(num_clusters_x());
+  const int k_atoms = (K + 63) / 64;
+  const int k_tiles = (k_atoms + 3) / 4;
+  const int num_m = (M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
+  const int num_n = (N + Cfg::BN - 1) / Cfg::BN;
+  const int num_tiles = num_m * num_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], 1);
+    }
+    for (int r = 0; r < R; ++r) mbar_init(&sf_ready[r], 8);  // 4 scale warps in each CTA of the pair
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * Cfg::EPI_WARPS);
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_mbarrier_init();
+  }
+  if (warp == Cfg::MMA_WARP) {
+    tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == Cfg::PRODUCER_WARP && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_sfa);
+    prefetch_tmap(&tmap_sfb);
+    prefetch_tmap(&tmap_c);
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == Cfg::PRODUCER_WARP) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int issued_last[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
+      int kc = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs) {
+        int tm, tn;
+        tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
+        for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+          const int s = kc % STAGES;
+          const uint32_t ph = static_cast<uint32_t>(kc / STAGES) & 1u;
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1u, abort_flag, status, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (Cfg::A_BYTES + Cfg::B_BYTES));
+          mbar_arrive_expect_tx(&sf_full[s], Cfg::SFA_BYTES + Cfg::SFB_BYTES);
+          const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0u);
+          tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tmap_a, bar, kt * Cfg::KTILE_BYTES,
+                           tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM);
+          tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tmap_b, bar, kt * Cfg::KTILE_BYTES,
+                           tn * Cfg::BN + static_cast<int>(rank) * 128);
+          tma_load_3d(sSFA + s * Cfg::SFA_BYTES, &tmap_sfa, &sf_full[s], 0, kt * 4, tm * 2 + static_cast<int>(rank));
+          tma_load_3d(sSFB + s * Cfg::SFB_BYTES, &tmap_sfb, &sf_full[s], 0, kt * 4, tn * 2);
+          issued_last[s] = kc;
+        }
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_last[s] >= 0) {
+            const uint32_t par = static_cast<uint32_t>(issued_last[s] / STAGES) & 1u;
+            mbar_wait_drain(&sf_full[s], par, status);
+            if (rank == 0) mbar_wait_drain(&full[s], par, status);
+          }
+      }
+    }
+  } else if (warp == Cfg::MMA_WARP) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (leader CTA only) ----------------
+      const uint32_t idesc = idesc_mxf4nvf4(2 * Cfg::BM, Cfg::BN);
+      const uint32_t t_acc = tmem_base;
+      const uint32_t acc_full_own = smem_u32(acc_full);
+      const uint32_t acc_full_peer = mapa_shared(acc_full_own, 1u);
+      bool ok = true;
+      int kc = 0, it = 0;
+      for (int t = pair; t < num_tiles && ok; t += npairs, ++it) {
+        if (!mbar_wait_cluster(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, status,
+                               kErrWaitAccEmpty)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+          const int s = kc % STAGES;
+          const int r = s;
+          if (!mbar_wait_cluster(&full[s], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
+                                 kErrWaitFull) ||
+              !mbar_wait_cluster(&sf_ready[r], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
+                                 kErrWaitFull + 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int na = min(4, k_atoms - kt * 4);
+          const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
+          const uint32_t t_sf = tmem_base + Cfg::TMEM_SF + r * Cfg::SF_COLS;
+          for (int j = 0; j < na; ++j)
+            mma_mxf4nvf4_pair(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j),
+                              idesc, t_sf + 4 * j, t_sf + 16 + 8 * j, (kt | j) != 0 ? 1u : 0u);
+          const uint32_t e_own = smem_u32(&empty[s]);
+          tc_commit_pair(e_own);
+          tc_commit_pair(mapa_shared(e_own, 1u));
+        }
+        if (!ok) break;
+        tc_commit_pair(acc_full_own);
+        tc_commit_pair(acc_full_peer);
+      }
+      if (!ok) {
+        tc_commit_pair(smem_u32(drain));
+        mbar_wait_drain(drain, 0u, status);
+      }
+    }
+  } else if (warp >= Cfg::SF_WARP0) {
+    // ---------------- scale warps (both CTAs): shared memory -> TMEM ----------------
+    const uint32_t quarter = static_cast<uint32_t>(warp & 3);
+    const int set = (warp - Cfg::SF_WARP0) >> 2;
+    const uint32_t sf_ready_leader0 = mapa_shared(smem_u32(&sf_ready[0]), 0u);
+    int kc = 0;
+    bool ok = true;
+    for (int t = pair; t < num_tiles && ok; t += npairs) {
+      for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+        if (kc % Cfg::SF_SETS != set) continue;
+        const int s = kc % STAGES;
+        const int r = s;
+        // the stage's scales have landed; the producer reloaded this stage only after
+        // the MMAs that last read region r had completed
+        if (!mbar_wait_cluster(&sf_full[s], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
+                               kErrWaitFull + 2)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint8_t* fa = sSFA + s * Cfg::SFA_BYTES + lane * 16;
+        const uint8_t* fb = sSFB + s * Cfg::SFB_BYTES + lane * 16;
+        uint32_t va[16], vb[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 a4 = *reinterpret_cast<const uint4*>(fa + j * Cfg::SF_ATOM);
+          va[4 * j] = a4.x;
+          va[4 * j + 1] = a4.y;
+          va[4 * j + 2] = a4.z;
+          va[4 * j + 3] = a4.w;
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const uint4 b4 = *reinterpret_cast<const uint4*>(fb + (g * 4 + j) * Cfg::SF_ATOM);
+            vb[8 * j + 4 * g] = b4.x;
+            vb[8 * j + 4 * g + 1] = b4.y;
+            vb[8 * j + 4 * g + 2] = b4.z;
+            vb[8 * j + 4 * g + 3] = b4.w;
+          }
+        }
+        const uint32_t t_sf = tmem_base + (quarter * 32u << 16) + Cfg::TMEM_SF + r * Cfg::SF_COLS;
+        tmem_st_32x32b_x16(t_sf, va);
+        tmem_st_32x32b_x32(t_sf + 16, vb);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive(&sf_ready[r]);
+          else
+            mbar_arrive_cluster(sf_ready_leader0 + r * 8u);
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 0-7, both CTAs) ----------------
+    constexpr int HALF = Cfg::BN / 2;
+    const int quarter = warp & 3, half = warp >> 2;
+    const float alpha = __fmul_rn(*a_gs, *b_gs);
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * HALF;
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0u);
+    uint8_t* box = sC + warp * Cfg::C_BOX_BYTES;
+    int it = 0;
+    bool stored = false;
+    for (int t = pair; t < num_tiles; t += npairs, ++it) {
+      int tm, tn;
+      tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
+      if (!mbar_wait_cluster(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, kErrWaitAccFull)) break;
+      tc_fence_after();
+      uint32_t p[HALF / 2];
+#pragma unroll
+      for (int c = 0; c < HALF; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_lane + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          p[c / 2 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[2 * i]), alpha),
+                                     __fmul_rn(__uint_as_float(v[2 * i + 1]), alpha));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+      const int row0 = tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM + quarter * 32;
+      const int col0 = tn * Cfg::BN + half * HALF;
+#pragma unroll
+      for (int chunk = 0; chunk < 2; ++chunk) {
+        // the previous TMA store from this box must have read it
+        if (stored) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+        }
+        // row `lane` of the 32 x 64 box, 128-byte swizzle: 16-byte unit u goes to u ^ (lane % 8)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int q = chunk * 32 + 4 * u;
+          *reinterpret_cast<uint4*>(box + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+              make_uint4(p[q], p[q + 1], p[q + 2], p[q + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < M && col0 + chunk * 64 < N) {
+          tma_store_2d(&tmap_c, box, col0 + chunk * 64, row0);
+          bulk_commit_group();
+        }
+        stored = true;
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+
+  // Both CTAs stay until the pair's last remote arrival and MMA are done.
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+  if (warp == Cfg::MMA_WARP) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------------
 
@@ -326,6 +658,90 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Swizzled scale buffer of `rows` rows viewed as [row groups][K atoms][128 words]:
+// box = 4 atoms (one K-tile) x `groups` row groups.  Out-of-range atoms/groups read 0.
+bool encode_sf_map(CUtensorMap* map, const uint8_t* sf, int64_t rows, int64_t K, int groups) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int64_t k_atoms = (K + 63) / 64;
+  const int64_t row_groups = (rows + 127) / 128;
+  const cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(k_atoms), static_cast<cuuint64_t>(row_groups)};
+  const cuuint64_t strides[2] = {512u, static_cast<cuuint64_t>(k_atoms * 512)};
+  const cuuint32_t box[3] = {128u, 4u, static_cast<cuuint32_t>(groups)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(sf), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int max_pair_clusters(int dev) {
+  static std::once_flag once[64];
+  static int clusters[64];
+  std::call_once(once[dev & 63], [&] {
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 148);
+    cfg.blockDim = dim3(PairCfg::THREADS);
+    cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel, &cfg) != cudaSuccess)
+      n = 0;
+    clusters[dev & 63] = n;
+  });
+  return clusters[dev & 63];
+}
+
+// BF16 output matrix, row stride ldc elements; box = 32 rows x 64 columns, 128-byte swizzle.
+bool encode_c_map(CUtensorMap* map, uint16_t* c, int64_t M, int64_t N, int64_t ldc) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldc * 2)};
+  const cuuint32_t box[2] = {64u, 32u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
+                        const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
+                        uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap ta, tb, tsa, tsb, tc;
+  if (!encode_codes_map(&ta, a_codes, M, K, 128) || !encode_codes_map(&tb, b_codes, N, K, 128) ||
+      !encode_sf_map(&tsa, a_sf, M, K, 1) || !encode_sf_map(&tsb, b_sf, N, K, 2) ||
+      !encode_c_map(&tc, c, M, N, ldc))
+    return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int max_clusters = max_pair_clusters(dev);
+  if (max_clusters <= 0) return cudaErrorLaunchOutOfResources;
+  const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(PairCfg::THREADS);
+  cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tb, tsa, tsb, tc, a_gs, b_gs, static_cast<int>(M),
+                            static_cast<int>(N), static_cast<int>(K), status);
+}
+
 template <int BN>
 cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* a_sf, const uint8_t* b_sf,
                         const float* a_gs, const float* b_gs, int64_t M, int64_t N, int64_t K, uint16_t* c,
@@ -354,6 +770,8 @@ cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint
 cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
                         uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream) {
+  if (M > 128 && N > 128)
+    return launch_pair(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status, stream);
   const int bn = N > 128 ? 256 : 128;
   CUtensorMap ta, tb;
   if (!encode_codes_map(&ta, a_codes, M, K, 128) || !encode_codes_map(&tb, b_codes, N, K, bn))
