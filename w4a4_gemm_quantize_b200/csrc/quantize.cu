@@ -164,8 +164,18 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
   const float d6 = __fmul_rn(6.0f, sg);
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const bool small = total < (int64_t(1) << 32);
   for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total; b += stride) {
-    const int64_t r = b / nblk, cb = b - r * nblk;
+    int64_t r, cb;
+    if (small) {
+      const uint32_t b32 = static_cast<uint32_t>(b), n32 = static_cast<uint32_t>(nblk);
+      const uint32_t r32 = b32 / n32;
+      r = r32;
+      cb = b32 - r32 * n32;
+    } else {
+      r = b / nblk;
+      cb = b - r * nblk;
+    }
     const uint16_t* src = x + r * ld + cb * 16;
     const uint4 lo = ld_nc_v4(src), hi = ld_nc_v4(src + 8);
     const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
@@ -191,12 +201,25 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
     if (MODE == 1) {
       const float factors[7] = {0.9f, 0.8f, 0.7f, 0.6f, 0.5f, 0.4f, 0.3f};
       uint32_t prev_s = best_s;
-#pragma unroll
+#pragma unroll 1
       for (int i = 0; i < 7; ++i) {
         const uint32_t s = cvt_e4m3_satfinite(__fmul_rn(factors[i], vb));
         if (s == prev_s) continue;  // same scale, same error: never a strict improvement
         prev_s = s;
         const float eff = __fmul_rn(e4m3_to_float(s), sg);
+        // Clip bound: if the block maximum lands above the 4|6 midpoint it is coded
+        // as 6, and its term alone makes e >= RN(d*d) with d = fma(-6, eff, amax_b):
+        // each fma of the error sum adds a non-negative term to a non-negative sum,
+        // and rounding is monotone.  Such a candidate cannot strictly improve when
+        // RN(d*d) >= best_e.  When d >= 0 (the maximum is clipped) later candidates,
+        // with smaller eff, have a larger d and cannot either, so the walk stops.
+        if (eff != 0.0f && __fmul_rn(amax_b, __frcp_rn(eff)) > 5.0f) {
+          const float d = __fmaf_rn(-6.0f, eff, amax_b);
+          if (__fmul_rn(d, d) >= best_e) {
+            if (d >= 0.0f) break;
+            continue;
+          }
+        }
         uint32_t c0, c1;
         encode_mags(ax, eff, c0, c1);
         const float e = block_sse(ax, c0, c1, eff);
