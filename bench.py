@@ -180,14 +180,21 @@ def barrier(world: int):
         dist.barrier()
 
 
-def max_over_ranks(value: float, world: int, device) -> float:
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device=device)
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, steps: int, flops_per_step: float, ms: float) -> float:
+    """Whole-job TFLOP/s under weak scaling: every rank runs `steps` steps of its own
+    problem, timed as the slowest rank's `ms`."""
+    return world * steps * flops_per_step / (ms * 1e-3) / 1e12
 
 
 # ------------------------------------------------------------------------------------------------
@@ -301,7 +308,7 @@ def run_ours(args, rank, world, local):
 
     flops, elems = work_units(cfg)
     peaks = load_peaks()
-    value = world * args.steps * flops / (ms * 1e-3) / 1e12
+    value = job_throughput(world, args.steps, flops, ms)
     step_ms = ms / args.steps
 
     # roofline of the dominant kernel: the first GEMM launch (M x N1 x K1)

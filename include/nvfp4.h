@@ -118,7 +118,9 @@ nvfp4_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, nvfp4
                               const float *global_scale, int64_t rows, int64_t cols, void *out,
                               int64_t ld_out, void *stream);
 
-/* Workspace nvfp4_gemm needs (device memory, any content on entry). */
+/* Workspace nvfp4_gemm needs (device memory, any content on entry): 256 bytes
+ * for the status word, plus, when M <= 32, room for the split-K partial tiles of
+ * the small-M kernel (counters and FP32 partials, about N * 128 * slices bytes). */
 size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Block-scaled W4A4 GEMM, C = (A s_a)(B s_b)^T * s_gA * s_gB, FP32 accumulation,
@@ -144,6 +146,15 @@ nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const f
  * NVFP4_ERR_CUDA if the copy fails.  Clears nothing: a workspace is reset by the
  * next nvfp4_gemm that uses it. */
 nvfp4_status nvfp4_read_device_error(const void *workspace, void *stream, uint32_t *word);
+
+/* Diagnostic for the bounded device-side waits (library plumbing; no
+ * counterpart on the pages).  Launches one thread that waits, with the same
+ * bounded wait the GEMM kernels use, on a barrier that nothing completes; after
+ * timeout_us microseconds (1 .. 2,000,000) it gives up and writes its status
+ * word into the first word of `workspace` (device, >= 256 bytes).  A following
+ * nvfp4_read_device_error(workspace, ...) must report NVFP4_ERR_TIMEOUT; the
+ * context stays usable.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA. */
+nvfp4_status nvfp4_selftest_wait_timeout(void *workspace, uint32_t timeout_us, void *stream);
 
 /* nvfp4_quantize for callers that cannot allocate device memory: a framework or
  * server plugin that owns no allocator and gets no workspace from its host, or a

@@ -80,7 +80,7 @@ def test_quantize_validation_before_any_cuda_call(lib):
 def test_gemm_validation_before_any_cuda_call(lib):
     P = ctypes.c_void_p
 
-    def g(M=16, N=16, K=64, ldc=16, ptr=16, ws=16, ws_bytes=256, gs=16):
+    def g(M=64, N=16, K=64, ldc=16, ptr=16, ws=16, ws_bytes=256, gs=16):
         p = P(ptr) if ptr else None
         return lib.nvfp4_gemm(p, p, P(gs), M, p, p, P(gs), N, K, p, ldc, P(ws) if ws else None, ws_bytes, None)
 
@@ -93,6 +93,11 @@ def test_gemm_validation_before_any_cuda_call(lib):
     assert g(ldc=20) == 3
     assert g(gs=2) == 3
     assert g() in (4, 5)
+    # small M uses split-K scratch after the status word: a 256-byte workspace is too small
+    need = lib.nvfp4_gemm_workspace_bytes(8, 14336, 4096)
+    assert need > 256
+    assert g(M=8, N=14336, ldc=14336, K=4096) == 7
+    assert g(M=8, N=14336, ldc=14336, K=4096, ws_bytes=need) in (4, 5)
 
 
 def test_dequantize_validation(lib):
@@ -105,3 +110,11 @@ def test_dequantize_validation(lib):
 
 def test_read_device_error_needs_workspace(lib):
     assert lib.nvfp4_read_device_error(None, None, None) == 1
+
+
+def test_selftest_validation(lib):
+    P = ctypes.c_void_p
+    assert lib.nvfp4_selftest_wait_timeout(None, 1000, None) == 1
+    assert lib.nvfp4_selftest_wait_timeout(P(16), 0, None) == 1
+    assert lib.nvfp4_selftest_wait_timeout(P(16), 3000000, None) == 1
+    assert lib.nvfp4_selftest_wait_timeout(P(8), 1000, None) == 3

@@ -49,7 +49,8 @@ def check(c_gpu, ref, absum, min_exact=0.9):
 def run_full(a, b, M, N, K):
     A, B = upload(*a), upload(*b)
     out = nv.nvfp4_gemm(A, B)
-    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    ws_bytes = nv.load_library().nvfp4_gemm_workspace_bytes(M, N, K)
+    ws = torch.full((ws_bytes,), 0xAB, dtype=torch.uint8, device="cuda")  # content on entry is arbitrary
     out2 = nv.nvfp4_gemm(A, B, workspace=ws)
     assert nv.read_device_error(ws) == 0
     assert torch.equal(out, out2)  # deterministic
@@ -81,6 +82,25 @@ def test_more_tiles_than_sms_full_compare(cuda_device, M, N, K):
     xa = workloads.activation(M, K, seed=M + 1, n_outlier_channels=2)
     xb = workloads.gaussian_weight(N, K, 0.02, seed=N + 1)
     run_full(oracle_operand(xa), oracle_operand(xb, oracle.SCALE_MSE), M, N, K)
+
+
+@pytest.mark.parametrize("M,N,K", [(24, 1000, 2080), (2, 384, 8192), (32, 14336, 512)])
+def test_small_m_split_k_full_compare(cuda_device, M, N, K):
+    """The small-M kernel (weights on the 128-row MMA side) with K split over several
+    CTAs: ragged N, a partial last K-tile, and the slice reduction."""
+    xa = workloads.activation(M, K, seed=M + 7, n_outlier_channels=2)
+    xb = workloads.gaussian_weight(N, K, 0.02, seed=N + 7)
+    run_full(oracle_operand(xa), oracle_operand(xb, oracle.SCALE_MSE), M, N, K)
+
+
+def test_bounded_wait_gives_up_and_reports(cuda_device):
+    """A device-side wait on a barrier nothing completes gives up after its limit,
+    writes its status word, and the context keeps working afterwards."""
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    nv.selftest_wait_timeout(ws, timeout_us=20000)
+    assert nv.read_device_error(ws) == 0x600
+    d = workloads.pr1(seed=0)
+    run_full(oracle_operand(d["x"]), oracle_operand(d["w"]), 16, 256, 256)
 
 
 def test_zero_and_sign_cases(cuda_device):

@@ -52,6 +52,7 @@ SIGNATURES = {
     "nvfp4_read_device_error": ([_P, _P, ctypes.POINTER(ctypes.c_uint32)], _I),
     "nvfp4_last_launch_count": ([], _I),
     "nvfp4_quantize_noalloc": ([_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P, _P, _P], _I),
+    "nvfp4_selftest_wait_timeout": ([_P, ctypes.c_uint32, _P], _I),
 }
 
 
@@ -212,6 +213,12 @@ def read_device_error(workspace: torch.Tensor, stream=None) -> int:
     if st not in (0, 6):
         _check(st, "nvfp4_read_device_error")
     return word.value
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, timeout_us: int = 20000, stream=None) -> None:
+    """Launch the bounded-wait diagnostic (see include/nvfp4.h); read the result with read_device_error."""
+    _check(load_library().nvfp4_selftest_wait_timeout(_ptr(workspace), timeout_us, _stream(stream)),
+           "nvfp4_selftest_wait_timeout")
 
 
 def last_launch_count() -> int:

@@ -157,7 +157,10 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, nvfp4
   return st;
 }
 
-size_t nvfp4_gemm_workspace_bytes(int64_t, int64_t, int64_t) { return kGemmWorkspace; }
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 1) return kGemmWorkspace;
+  return kGemmWorkspace + nvfp4::gemm_scratch_bytes(M, N, K);
+}
 
 nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale, int64_t M,
                         const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale, int64_t N,
@@ -167,7 +170,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const f
   if (K % 32 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return NVFP4_ERR_SHAPE;
   if (!a_codes || !a_scales || !a_global_scale || !b_codes || !b_scales || !b_global_scale || !c)
     return NVFP4_ERR_INVALID_ARG;
-  if (!workspace || workspace_bytes < kGemmWorkspace) return NVFP4_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < nvfp4_gemm_workspace_bytes(M, N, K)) return NVFP4_ERR_WORKSPACE;
   if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) ||
       !aligned16(c) || !aligned16(workspace) || ldc % 8 != 0 ||
       (reinterpret_cast<uintptr_t>(a_global_scale) & 3u) || (reinterpret_cast<uintptr_t>(b_global_scale) & 3u))
@@ -193,6 +196,19 @@ nvfp4_status nvfp4_read_device_error(const void* workspace, void* stream, uint32
   if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (word) *word = w;
   return w == 0 ? NVFP4_OK : NVFP4_ERR_TIMEOUT;
+}
+
+nvfp4_status nvfp4_selftest_wait_timeout(void* workspace, uint32_t timeout_us, void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (!workspace || timeout_us == 0 || timeout_us > 2000000u) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+  nvfp4_status st = check_device_cached();
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  st = from_cuda(nvfp4::launch_selftest_wait(static_cast<uint32_t*>(workspace), uint64_t(timeout_us) * 1000u, s));
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
 }
 
 // Kernels the most recent call on this thread enqueued (benchmark bookkeeping).

@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       int tm, tn;
       tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
-      if (!mbar_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, kErrWaitAccFull)) break;
+      if (!warp_wait(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, kErrWaitAccFull)) break;
       tc_fence_after();
       uint32_t p[HALF / 2];
 #pragma unroll
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         const int r = s;
         // the stage's scales have landed; the producer reloaded this stage only after
         // the MMAs that last read region r had completed
-        if (!mbar_wait_cluster(&sf_full[s], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
+        if (!warp_wait_cluster(&sf_full[s], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
                                kErrWaitFull + 2)) {
           ok = false;
           break;
@@ -570,7 +570,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     for (int t = pair; t < num_tiles; t += npairs, ++it) {
       int tm, tn;
       tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
-      if (!mbar_wait_cluster(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, kErrWaitAccFull)) break;
+      if (!warp_wait_cluster(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, kErrWaitAccFull)) break;
       tc_fence_after();
       uint32_t p[HALF / 2];
 #pragma unroll
@@ -626,8 +626,218 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------------------------
+// Decode kernel (M <= 32): weights on the 128-row side of the MMA, split-K
+// ---------------------------------------------------------------------------------------------
+//
+// For a handful of activation rows the GEMM is a stream over the weights, so the
+// weight matrix B takes the MMA's 128-row A slot (D^T = B A^T, 128 x 32 x 64 per
+// instruction) and each CTA handles one 128-row weight tile over a slice of K.
+// Partial FP32 tiles go to the workspace; the last CTA of a weight tile (by an
+// atomic counter) sums the slices in slice order, applies s_gA s_gB and writes
+// C (transposed back) in BF16, so the result does not depend on arrival order.
+
+struct DecodeCfg {
+  static constexpr int BM = 128;                 // weight rows per CTA
+  static constexpr int BN = 32;                  // activation rows (padded)
+  static constexpr int KTILE_BYTES = 128;
+  static constexpr int A_BYTES = BM * KTILE_BYTES;   // 16 KB of weight codes
+  static constexpr int B_BYTES = BN * KTILE_BYTES;   // 4 KB of activation codes
+  static constexpr int SF_ATOM = 512;
+  static constexpr int SFA_BYTES = 4 * SF_ATOM;
+  static constexpr int SFB_BYTES = 4 * SF_ATOM;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = 4;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+  static constexpr int THREADS = 192;            // warps 0-3 epilogue, 4 producer, 5 MMA
+  static constexpr int TMEM_SF = 32;             // two scale regions of 32 columns after the accumulator
+  static constexpr int TMEM_COLS = 128;
+};
+
+__global__ void __launch_bounds__(DecodeCfg::THREADS)
+    gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                       const uint8_t* __restrict__ sf_w, const uint8_t* __restrict__ sf_x,
+                       const float* __restrict__ a_gs, const float* __restrict__ b_gs, uint16_t* __restrict__ C,
+                       int M, int N, int K, int64_t ldc, int splits, float* __restrict__ partial,
+                       uint32_t* __restrict__ counters, uint32_t* __restrict__ status) {
+  using Cfg = DecodeCfg;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * Cfg::A_BYTES;
+  uint8_t* sSFA = sB + STAGES * Cfg::B_BYTES;
+  uint8_t* sSFB = sSFA + STAGES * Cfg::SFA_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * Cfg::SFB_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* last_flag = tmem_slot + 2;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x / splits, split = blockIdx.x - tile * splits;
+  const int k_atoms = (K + 63) / 64;
+  const int k_tiles = (k_atoms + 3) / 4;
+  const int kt0 = static_cast<int>(static_cast<int64_t>(split) * k_tiles / splits);
+  const int kt1 = static_cast<int>(static_cast<int64_t>(split + 1) * k_tiles / splits);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_mbarrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_x);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      int issued_last[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
+      for (int kt = kt0, i = 0; kt < kt1; ++kt, ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&empty[s], (static_cast<uint32_t>(i / STAGES) & 1u) ^ 1u, abort_flag, status, kErrWaitEmpty))
+          break;
+        const int ka0 = kt * 4;
+        const int na = min(4, k_atoms - ka0);
+        const uint32_t sf_bytes = static_cast<uint32_t>(na) * Cfg::SF_ATOM;
+        mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + 2 * sf_bytes);
+        tma_load_2d(sA + s * Cfg::A_BYTES, &tmap_w, &full[s], kt * Cfg::KTILE_BYTES, tile * Cfg::BM);
+        tma_load_2d(sB + s * Cfg::B_BYTES, &tmap_x, &full[s], kt * Cfg::KTILE_BYTES, 0);
+        bulk_load(sSFA + s * Cfg::SFA_BYTES, sf_w + (static_cast<size_t>(tile) * k_atoms + ka0) * Cfg::SF_ATOM,
+                  sf_bytes, &full[s]);
+        bulk_load(sSFB + s * Cfg::SFB_BYTES, sf_x + static_cast<size_t>(ka0) * Cfg::SF_ATOM, sf_bytes, &full[s]);
+        issued_last[s] = i;
+      }
+      if (*abort_flag)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_last[s] >= 0)
+            mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_last[s] / STAGES) & 1u, status);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_mxf4nvf4(Cfg::BM, Cfg::BN);
+      bool ok = true;
+      for (int kt = kt0, i = 0; kt < kt1; ++kt, ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&full[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int na = min(4, k_atoms - kt * 4);
+        const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
+        const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
+        const uint32_t sfa_base = smem_u32(sSFA + s * Cfg::SFA_BYTES);
+        const uint32_t sfb_base = smem_u32(sSFB + s * Cfg::SFB_BYTES);
+        const uint32_t t_sf = tmem_base + Cfg::TMEM_SF + (i & 1) * 32;
+        for (int j = 0; j < na; ++j) {
+          tc_cp_sf(t_sf + 4 * j, sdesc_sf_tile(sfa_base + j * Cfg::SF_ATOM));
+          tc_cp_sf(t_sf + 16 + 4 * j, sdesc_sf_tile(sfb_base + j * Cfg::SF_ATOM));
+          mma_mxf4nvf4(tmem_base, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
+                       t_sf + 4 * j, t_sf + 16 + 4 * j, (i | j) != 0 ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+      }
+      if (ok) {
+        tc_commit(acc_full);
+      } else {
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0u, status);
+      }
+    }
+  } else {
+    // epilogue: lane = weight row n of the tile, 32 columns = activation rows m
+    const int n = tile * Cfg::BM + warp * 32 + lane;
+    warp_wait(acc_full, 0u, abort_flag, status, kErrWaitAccFull);
+    // one decision for all four warps (they meet at the named barrier below)
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (threadIdx.x == 0) *last_flag = *abort_flag ? 0u : 2u;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const bool have = *last_flag == 2u;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    uint32_t v[32];
+    if (have) {
+      tc_fence_after();
+      tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16), v);
+      tmem_ld_wait();
+    }
+    const float alpha = __fmul_rn(*a_gs, *b_gs);
+    if (have && splits == 1) {
+      if (n < N)
+        for (int m = 0; m < M; ++m)
+          C[static_cast<int64_t>(m) * ldc + n] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__uint_as_float(v[m]), alpha)));
+    } else if (have) {
+      // this slice's partial tile, then the last slice to finish reduces all of them
+      float4* dst = reinterpret_cast<float4*>(partial + ((static_cast<int64_t>(split) * N + n) * Cfg::BN));
+      if (n < N)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+                               __uint_as_float(v[4 * i + 3]));
+      __threadfence();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 0) *last_flag = (atomicAdd(&counters[tile], 1u) == static_cast<uint32_t>(splits - 1)) ? 1u : 0u;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (*last_flag) {
+        __threadfence();
+        if (n < N) {
+          float acc[32];
+#pragma unroll
+          for (int m = 0; m < 32; ++m) acc[m] = 0.0f;
+          for (int sp = 0; sp < splits; ++sp) {
+            const float4* src = reinterpret_cast<const float4*>(partial + ((static_cast<int64_t>(sp) * N + n) * Cfg::BN));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 f = __ldcg(src + i);
+              acc[4 * i] = __fadd_rn(acc[4 * i], f.x);
+              acc[4 * i + 1] = __fadd_rn(acc[4 * i + 1], f.y);
+              acc[4 * i + 2] = __fadd_rn(acc[4 * i + 2], f.z);
+              acc[4 * i + 3] = __fadd_rn(acc[4 * i + 3], f.w);
+            }
+          }
+          for (int m = 0; m < M; ++m)
+            C[static_cast<int64_t>(m) * ldc + n] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(acc[m], alpha)));
+        }
+        if (threadIdx.x == 0) counters[tile] = 0u;  // ready for the next call
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------------
+
+// Decode workspace after the 256-byte status block: one counter per 128-row
+// weight tile (rounded up to 256 bytes), then the FP32 partial tiles.
+size_t decode_counter_bytes(int64_t N) { return static_cast<size_t>(((N + 127) / 128 * 4 + 255) / 256 * 256); }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -742,6 +952,46 @@ cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float
                             static_cast<int>(N), static_cast<int>(K), status);
 }
 
+// Slices of K per 128-row weight tile: as many as fit in one wave of two CTAs per SM.
+int decode_splits(int64_t N, int64_t K, int sms) {
+  const int64_t tiles = (N + 127) / 128;
+  const int64_t k_tiles = (K + 255) / 256;
+  int64_t s = 2 * static_cast<int64_t>(sms) / tiles;
+  if (s > k_tiles / 2) s = k_tiles / 2;
+  if (s > 16) s = 16;
+  return static_cast<int>(s < 1 ? 1 : s);
+}
+
+cudaError_t launch_decode(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
+                          const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
+                          uint16_t* c, int64_t ldc, uint32_t* status, uint8_t* scratch, cudaStream_t stream) {
+  CUtensorMap tw, tx;
+  if (!encode_codes_map(&tw, b_codes, N, K, 128) || !encode_codes_map(&tx, a_codes, M, K, DecodeCfg::BN))
+    return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static std::once_flag once[64];
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(once[dev & 63], [&] {
+    attr_err = cudaFuncSetAttribute(gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    DecodeCfg::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int tiles = static_cast<int>((N + 127) / 128);
+  const int splits = decode_splits(N, K, sms);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(scratch);
+  float* partial = reinterpret_cast<float*>(scratch + decode_counter_bytes(N));
+  if (splits > 1) {
+    cudaError_t e = cudaMemsetAsync(counters, 0, static_cast<size_t>(tiles) * 4, stream);
+    if (e != cudaSuccess) return e;
+  }
+  gemm_decode_kernel<<<tiles * splits, DecodeCfg::THREADS, DecodeCfg::SMEM_BYTES, stream>>>(
+      tw, tx, b_sf, a_sf, a_gs, b_gs, c, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), ldc, splits,
+      partial, counters, status);
+  return cudaGetLastError();
+}
+
 template <int BN>
 cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* a_sf, const uint8_t* b_sf,
                         const float* a_gs, const float* b_gs, int64_t M, int64_t N, int64_t K, uint16_t* c,
@@ -767,9 +1017,18 @@ cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint
 
 }  // namespace
 
+size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M > DecodeCfg::BN) return 0;
+  const int splits = decode_splits(N, K, 148 * 2);  // upper bound over SM counts up to 296
+  return decode_counter_bytes(N) + static_cast<size_t>(splits) * N * DecodeCfg::BN * 4;
+}
+
 cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
                         uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream) {
+  if (M <= DecodeCfg::BN)
+    return launch_decode(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status,
+                         reinterpret_cast<uint8_t*>(status) + 256, stream);
   if (M > 128 && N > 128)
     return launch_pair(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status, stream);
   const int bn = N > 128 ? 256 : 128;

@@ -18,11 +18,18 @@ cudaError_t launch_sf_pad_zero(uint8_t* scales, int64_t rows, int64_t nblk, cuda
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, bool swizzled, const float* gs,
                               int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out, cudaStream_t stream);
 
+// Bounded-wait self test (quantize.cu).
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t stream);
+
 // GEMM launcher (gemm_sm100.cu).  Returns cudaErrorInvalidValue when a tensor
 // map cannot be encoded.
 cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
                         uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream);
+
+// Bytes the GEMM needs in its workspace after the 256-byte status block
+// (split-K partial tiles of the small-M kernel); 0 when none.
+size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 
 // Number of kernel launches the last call of each entry point enqueued (for
 // the benchmark's launch count); host-side bookkeeping only.

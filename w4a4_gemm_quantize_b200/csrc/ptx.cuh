@@ -21,6 +21,7 @@ enum : uint32_t {
   kErrWaitAccFull = 0x300,   // epilogue waiting for the accumulator
   kErrWaitAccEmpty = 0x400,  // MMA issuer waiting for the epilogue to drain TMEM
   kErrWaitDrain = 0x500,     // teardown waiting for in-flight copies / MMAs
+  kErrSelfTest = 0x600,      // the wait of nvfp4_selftest_wait_timeout (expected to give up)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -72,7 +73,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 // timeout it raises *abort and records `where` in the device status word.
 // Returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
-                                          uint32_t* status, uint32_t where) {
+                                          uint32_t* status, uint32_t where, uint64_t timeout_ns = kWaitTimeoutNs) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -80,7 +81,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(addr, parity)) return true;
     if ((n & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > timeout_ns) {
         *abort = 1u;
         if (status) atomicCAS(status, 0u, where);
         return false;
@@ -284,6 +285,19 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
       }
     }
   }
+}
+
+// Warp-uniform waits: every lane polls, then the warp votes, so all lanes take the
+// same branch (the .sync.aligned tcgen05 instructions that follow need the whole
+// warp) even if a bounded wait gives up while another lane sees the phase complete.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort, uint32_t* status,
+                                          uint32_t where) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort, status, where)) != 0;
+}
+
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
+                                                  uint32_t* status, uint32_t where) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait_cluster(bar, parity, abort, status, where)) != 0;
 }
 
 // Pair TMA loads: the data lands in this CTA's shared memory, the completed bytes

@@ -94,51 +94,89 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
   }
 }
 
-// Magnitude codes of 16 values for effective scale eff (eff == 0: all zero).
-__device__ __forceinline__ void encode_mags(const float (&ax)[16], float eff, uint32_t& c0, uint32_t& c1) {
-  if (eff == 0.0f) {
-    c0 = c1 = 0u;
+// Two binary32 values in one 64-bit register (element 2i low, 2i+1 high) for the
+// packed f32x2 arithmetic of sm_100.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// RN32(a * b) on both halves.
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// RN32(a * b + c) on both halves (one rounding each).
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// Sign bit of each of the 16 values moved to bit 3 of its code nibble.
+__device__ __forceinline__ void sign_codes(const uint64_t (&x2)[8], uint32_t& c0, uint32_t& c1) {
+  c0 = c1 = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t lo = static_cast<uint32_t>(x2[i]) >> 31, hi = static_cast<uint32_t>(x2[i] >> 32) >> 31;
+    const uint32_t nib = (lo << 3) | (hi << 7);
+    if (i < 4)
+      c0 |= nib << (8 * i);
+    else
+      c1 |= nib << (8 * (i - 4));
+  }
+}
+
+// Signed 4-bit codes of 16 values (packed pairs x2) for effective scale eff:
+// y = RN32(x * RN32(1/eff)) rounded to the E2M1 grid (RNE, saturating), the sign
+// of x kept by the conversion (-0 and small negatives give code 0x8).
+__device__ __forceinline__ void encode_codes(const uint64_t (&x2)[8], float eff, uint32_t& c0, uint32_t& c1) {
+  if (eff == 0.0f) {  // zero scale: every magnitude is 0, only the signs remain
+    sign_codes(x2, c0, c1);
     return;
   }
   const float r = __frcp_rn(eff);
+  const uint64_t r2 = pack2(r, r);
   float y[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) y[k] = __fmul_rn(ax[k], r);
+  for (int i = 0; i < 8; ++i) unpack2(mul2(x2[i], r2), y[2 * i], y[2 * i + 1]);
   if (isinf(r)) {
-    // 1/eff overflowed: a zero input gives 0 * inf = NaN; it encodes as 0.
+    // 1/eff overflowed: +-0 * inf is NaN; a zero input keeps its own (signed) zero
 #pragma unroll
-    for (int k = 0; k < 16; ++k) y[k] = fmaxf(y[k], 0.0f);
+    for (int i = 0; i < 8; ++i) {
+      float lo, hi;
+      unpack2(x2[i], lo, hi);
+      if (lo == 0.0f) y[2 * i] = lo;
+      if (hi == 0.0f) y[2 * i + 1] = hi;
+    }
   }
   c0 = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
   c1 = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
 }
 
-// Squared reconstruction error of the block, accumulated in element order.
-__device__ __forceinline__ float block_sse(const float (&ax)[16], uint32_t c0, uint32_t c1, float eff) {
+// Squared reconstruction error of the block in element order:
+// d_k = RN32(x_k - q_k * eff) (one fma), e = fma(d_k, d_k, e), k = 0..15.
+__device__ __forceinline__ float block_sse(const uint64_t (&x2)[8], uint32_t c0, uint32_t c1, float eff) {
+  const uint64_t neff2 = pack2(-eff, -eff);
   float e = 0.0f;
 #pragma unroll
-  for (int w = 0; w < 2; ++w) {
-    const uint32_t word = w ? c1 : c0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t h2 = e2m1x2_to_half2(word, k);
-      const float q_lo = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFFu)));
-      const float q_hi = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 >> 16)));
-      const float d0 = __fmaf_rn(-q_lo, eff, ax[8 * w + 2 * k]);
-      e = __fmaf_rn(d0, d0, e);
-      const float d1 = __fmaf_rn(-q_hi, eff, ax[8 * w + 2 * k + 1]);
-      e = __fmaf_rn(d1, d1, e);
-    }
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t h2 = e2m1x2_to_half2(i < 4 ? c0 : c1, i & 3);
+    const float q_lo = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFFu)));
+    const float q_hi = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 >> 16)));
+    float d_lo, d_hi;
+    unpack2(fma2(pack2(q_lo, q_hi), neff2, x2[i]), d_lo, d_hi);
+    e = __fmaf_rn(d_lo, d_lo, e);
+    e = __fmaf_rn(d_hi, d_hi, e);
   }
   return e;
-}
-
-// Sign bits of eight BF16 values (words w0..w3, two values each) moved to bit 3
-// of their nibble in a packed code word.
-__device__ __forceinline__ uint32_t sign_nibbles(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
-  return ((w0 >> 12) & 0x8u) | ((w0 >> 24) & 0x80u) | ((w1 >> 4) & 0x800u) | ((w1 >> 16) & 0x8000u) |
-         ((w2 << 4) & 0x80000u) | ((w2 >> 8) & 0x800000u) | ((w3 << 12) & 0x8000000u) |
-         (w3 & 0x80000000u);
 }
 
 __device__ __forceinline__ int64_t swizzled_offset(int64_t r, int64_t c, int64_t atoms_per_group) {
@@ -151,8 +189,10 @@ __device__ __forceinline__ float global_scale(const float* gs_in, const uint32_t
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
 
+// Absmax blocks are memory-bound: ask for high occupancy (6 CTAs of 256 threads per
+// SM) so that more loads are in flight; the MSE search is arithmetic-bound.
 template <int MODE, bool SWZ>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(
+__global__ void __launch_bounds__(kThreads, MODE == 0 ? 6 : 4) quantize_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, const float* __restrict__ gs_in,
     const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ gs_out, float* __restrict__ block_err) {
@@ -165,8 +205,18 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const bool small = total < (int64_t(1) << 32);
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total; b += stride) {
-    int64_t r, cb;
+  // When a row's block count is a multiple of 4, four consecutive blocks (lanes
+  // 4j..4j+3) own four consecutive bytes of the swizzled scale layout.
+  const bool pack_scales = SWZ && (nblk & 3) == 0;
+  const int lane = threadIdx.x & 31;
+  // warp-uniform loop: every lane of a warp runs the same iterations
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31); base < total;
+       base += stride) {
+    const int64_t b = base + lane;
+    const bool active = b < total;
+    int64_t r = 0, cb = 0;
+    uint32_t best_s = 0;
+    if (active) {
     if (small) {
       const uint32_t b32 = static_cast<uint32_t>(b), n32 = static_cast<uint32_t>(nblk);
       const uint32_t r32 = b32 / n32;
@@ -179,24 +229,23 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
     const uint16_t* src = x + r * ld + cb * 16;
     const uint4 lo = ld_nc_v4(src), hi = ld_nc_v4(src + 8);
     const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-    float ax[16];
+    uint64_t x2[8];  // the block as signed binary32 pairs (BF16 widening is exact)
     uint32_t mb = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      ax[2 * i] = bf16_bits_to_float(w[i] & 0x7FFFu);
-      ax[2 * i + 1] = bf16_bits_to_float((w[i] >> 16) & 0x7FFFu);
+      x2[i] = pack2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
       mb = __vmaxu2(mb, w[i] & 0x7FFF7FFFu);
     }
     const float amax_b = bf16_bits_to_float(max(mb & 0xFFFFu, mb >> 16));
     const float vb = __fdiv_rn(amax_b, d6);
 
     // candidate f = 1: the absmax scale
-    uint32_t best_s = cvt_e4m3_satfinite(vb);
+    best_s = cvt_e4m3_satfinite(vb);
     float best_eff = __fmul_rn(e4m3_to_float(best_s), sg);
     uint32_t best_c0, best_c1;
-    encode_mags(ax, best_eff, best_c0, best_c1);
+    encode_codes(x2, best_eff, best_c0, best_c1);
     float best_e = 0.0f;
-    if (MODE == 1 || block_err) best_e = block_sse(ax, best_c0, best_c1, best_eff);
+    if (MODE == 1 || block_err) best_e = block_sse(x2, best_c0, best_c1, best_eff);
 
     if (MODE == 1) {
       const float factors[7] = {0.9f, 0.8f, 0.7f, 0.6f, 0.5f, 0.4f, 0.3f};
@@ -221,8 +270,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
           }
         }
         uint32_t c0, c1;
-        encode_mags(ax, eff, c0, c1);
-        const float e = block_sse(ax, c0, c1, eff);
+        encode_codes(x2, eff, c0, c1);
+        const float e = block_sse(x2, c0, c1, eff);
         if (e < best_e) {
           best_e = e;
           best_s = s;
@@ -232,14 +281,23 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
       }
     }
 
-    best_c0 |= sign_nibbles(w[0], w[1], w[2], w[3]);
-    best_c1 |= sign_nibbles(w[4], w[5], w[6], w[7]);
     *reinterpret_cast<uint2*>(codes + r * (cols / 2) + cb * 8) = make_uint2(best_c0, best_c1);
-    if (SWZ)
-      scales[swizzled_offset(r, cb, atoms_per_group)] = static_cast<uint8_t>(best_s);
-    else
-      scales[b] = static_cast<uint8_t>(best_s);
+    if (!pack_scales) {
+      if (SWZ)
+        scales[swizzled_offset(r, cb, atoms_per_group)] = static_cast<uint8_t>(best_s);
+      else
+        scales[b] = static_cast<uint8_t>(best_s);
+    }
     if (block_err) block_err[b] = best_e;
+    }  // active
+    if (pack_scales) {
+      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, best_s, 1);
+      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, best_s, 2);
+      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, best_s, 3);
+      if (active && (cb & 3) == 0)
+        *reinterpret_cast<uint32_t*>(scales + swizzled_offset(r, cb, atoms_per_group)) =
+            best_s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    }
   }
 }
 
@@ -305,6 +363,19 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const uint8_t* __r
   }
 }
 
+// One thread waits, with the kernels' bounded wait, on an mbarrier that nothing
+// completes; it gives up after timeout_ns and records kErrSelfTest.
+__global__ void selftest_wait_kernel(uint32_t* status, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0u;
+    fence_mbarrier_init();
+    mbar_wait(&bar, 0u, &abort_flag, status, kErrSelfTest, timeout_ns);
+  }
+}
+
 int grid_for(int64_t work, int threads) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -352,6 +423,11 @@ cudaError_t launch_sf_pad_zero(uint8_t* scales, int64_t rows, int64_t nblk, cuda
   const int64_t pads = (rp - rows) * cp + rows * (cp - nblk);
   if (pads == 0) return cudaSuccess;
   sf_pad_zero_kernel<<<grid_for(pads, kThreads), kThreads, 0, stream>>>(scales, rows, nblk);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(status, timeout_ns);
   return cudaGetLastError();
 }
 
