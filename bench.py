@@ -56,10 +56,16 @@ def parse_args():
     return p.parse_args()
 
 
-def source_hash() -> str:
+KERNEL_SOURCES = {"gemm": ["gemm_sm100.cu", "ptx.cuh", "internal.h"],
+                  "quantize": ["quantize.cu", "ptx.cuh", "internal.h"]}
+
+
+def source_hash(kernel: str = "gemm") -> str:
+    """Hash of the source files a kernel is built from (ncu summaries record it, so
+    counters taken on an older kernel are never reported for a newer one)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "w4a4_gemm_quantize_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -87,7 +93,7 @@ def profiled_traffic(kernel: str, workload: str):
             if ":" in line and line.startswith("- "):
                 k, v = line[2:].split(":", 1)
                 vals[k.strip()] = v.strip().strip("`")
-    if vals.get("source_hash") != source_hash():
+    if vals.get("source_hash") != source_hash(kernel):
         return None
     try:
         return float(vals["traffic_bytes_per_launch"])

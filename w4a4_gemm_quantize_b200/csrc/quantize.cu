@@ -33,9 +33,10 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// Streaming 16-byte load: read-only path, no L1 allocation, 256-byte L2 fetches.
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
@@ -189,10 +190,8 @@ __device__ __forceinline__ float global_scale(const float* gs_in, const uint32_t
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
 
-// Absmax blocks are memory-bound: ask for high occupancy (6 CTAs of 256 threads per
-// SM) so that more loads are in flight; the MSE search is arithmetic-bound.
 template <int MODE, bool SWZ>
-__global__ void __launch_bounds__(kThreads, MODE == 0 ? 6 : 4) quantize_kernel(
+__global__ void __launch_bounds__(kThreads) quantize_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, const float* __restrict__ gs_in,
     const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ gs_out, float* __restrict__ block_err) {
