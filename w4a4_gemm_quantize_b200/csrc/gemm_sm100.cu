@@ -316,7 +316,10 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 // the 4-way replication the block-scaled MMA reads.  This keeps the copy off the
 // tensor pipe (tcgen05.cp of the same bytes, even one copy per MMA, serialises with
 // the MMAs).  Three sets rotate over K-tiles so that one set's barrier round trip
-// overlaps the others' copies.  A stage's region is free again when its
+// overlaps the others' copies.  The leader's set also waits for the stage's A/B
+// bytes before it arrives, so the MMA issuer waits on one barrier per K-tile: every
+// wait in the issuing thread lets the tensor pipe's queue run dry, and with four
+// MMAs per wait that costs a tenth of the pipe's time per extra wait.  A stage's region is free again when its
 // shared-memory slot is: the producer reloads stage s only after the MMAs that
 // read it completed, so no separate release barrier is needed.
 //
@@ -463,7 +466,6 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       const uint32_t idesc = idesc_mxf4nvf4(2 * Cfg::BM, Cfg::BN);
       const uint32_t t_acc = tmem_base;
       const uint32_t acc_full_own = smem_u32(acc_full);
-      const uint32_t acc_full_peer = mapa_shared(acc_full_own, 1u);
       bool ok = true;
       int kc = 0, it = 0;
       for (int t = pair; t < num_tiles && ok; t += npairs, ++it) {
@@ -476,9 +478,9 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
           const int s = kc % STAGES;
           const int r = s;
-          if (!mbar_wait_cluster(&full[s], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
-                                 kErrWaitFull) ||
-              !mbar_wait_cluster(&sf_ready[r], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
+          // one wait per K-tile: the leader's scale warps arrive on sf_ready only after
+          // they have also seen the stage's A/B bytes land on full[s]
+          if (!mbar_wait_cluster(&sf_ready[r], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
                                  kErrWaitFull + 1)) {
             ok = false;
             break;
@@ -491,13 +493,10 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           for (int j = 0; j < na; ++j)
             mma_mxf4nvf4_pair(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j),
                               idesc, t_sf + 4 * j, t_sf + 16 + 8 * j, (kt | j) != 0 ? 1u : 0u);
-          const uint32_t e_own = smem_u32(&empty[s]);
-          tc_commit_pair(e_own);
-          tc_commit_pair(mapa_shared(e_own, 1u));
+          tc_commit_pair_both(smem_u32(&empty[s]));
         }
         if (!ok) break;
-        tc_commit_pair(acc_full_own);
-        tc_commit_pair(acc_full_peer);
+        tc_commit_pair_both(acc_full_own);
       }
       if (!ok) {
         tc_commit_pair(smem_u32(drain));
@@ -547,13 +546,18 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         tmem_st_32x32b_x16(t_sf, va);
         tmem_st_32x32b_x32(t_sf + 16, vb);
         tmem_st_wait();
+        if (rank == 0 && !warp_wait_cluster(&full[s], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
+                                            kErrWaitFull)) {
+          ok = false;
+          break;
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           if (rank == 0)
             mbar_arrive(&sf_ready[r]);
           else
-            mbar_arrive_cluster(sf_ready_leader0 + r * 8u);
+            mbar_arrive_cluster_relaxed(sf_ready_leader0 + r * 8u);
         }
       }
     }
@@ -585,7 +589,12 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(acc_empty);
+        else
+          mbar_arrive_cluster_relaxed(acc_empty_leader);
+      }
       const int row0 = tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM + quarter * 32;
       const int col0 = tn * Cfg::BN + half * HALF;
 #pragma unroll

@@ -256,6 +256,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Relaxed arrive on an mbarrier that may live in the other CTA.  For a thread whose
+// only work before the arrive is tensor-memory traffic it has already waited for
+// (tcgen05.wait::st / wait::ld, then tcgen05.fence::before_thread_sync): there are
+// no generic-proxy writes to publish, and a cluster-scope release costs about as much
+// as a K-tile of MMAs.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
   uint32_t done;
   asm volatile(
@@ -340,6 +349,18 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster_addr) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    bar_cluster_addr)
                : "memory");
+}
+
+// One commit whose arrival goes to the mbarrier at the same shared-memory offset
+// in both CTAs of the pair (`bar` is this CTA's copy).  This signals barriers only:
+// no data moves.  One commit instead of two halves the commit traffic of the
+// tensor pipe.
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
 }
 
 // 256 x N x 64 block-scaled MMA over the CTA pair: rows 0-127 from the leader's
