@@ -135,20 +135,20 @@ __device__ __forceinline__ void sign_codes(const uint64_t (&x2)[8], uint32_t& c0
   }
 }
 
-// Signed 4-bit codes of 16 values (packed pairs x2) for effective scale eff:
-// y = RN32(x * RN32(1/eff)) rounded to the E2M1 grid (RNE, saturating), the sign
-// of x kept by the conversion (-0 and small negatives give code 0x8).
-__device__ __forceinline__ void encode_codes(const uint64_t (&x2)[8], float eff, uint32_t& c0, uint32_t& c1) {
+// Signed 4-bit codes of 16 values (packed pairs x2) for effective scale eff with
+// rcp = RN32(1/eff): y = RN32(x * rcp) rounded to the E2M1 grid (RNE, saturating),
+// the sign of x kept by the conversion (-0 and small negatives give code 0x8).
+__device__ __forceinline__ void encode_codes(const uint64_t (&x2)[8], float eff, float rcp, uint32_t& c0,
+                                             uint32_t& c1) {
   if (eff == 0.0f) {  // zero scale: every magnitude is 0, only the signs remain
     sign_codes(x2, c0, c1);
     return;
   }
-  const float r = __frcp_rn(eff);
-  const uint64_t r2 = pack2(r, r);
+  const uint64_t r2 = pack2(rcp, rcp);
   float y[16];
 #pragma unroll
   for (int i = 0; i < 8; ++i) unpack2(mul2(x2[i], r2), y[2 * i], y[2 * i + 1]);
-  if (isinf(r)) {
+  if (isinf(rcp)) {
     // 1/eff overflowed: +-0 * inf is NaN; a zero input keeps its own (signed) zero
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -190,112 +190,129 @@ __device__ __forceinline__ float global_scale(const float* gs_in, const uint32_t
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
 
+// The 127 finite non-negative E4M3 scale bytes of one tensor, decoded: eff =
+// RN32(dec(s) s_g) and RN32(1/eff) (0 for eff = 0).  Every CTA builds them once, so
+// each candidate scale costs two shared-memory reads instead of a conversion, a
+// product and a correctly rounded reciprocal.
+struct ScaleTables {
+  float eff[128];
+  float rcp[128];
+};
+
+// One warp handles 32 consecutive blocks of one row (lane = block); warps walk a
+// fixed column chunk down the rows, so block coordinates and output offsets need
+// no division.
 template <int MODE, bool SWZ>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(
+__global__ void __launch_bounds__(kThreads, MODE == 1 ? 4 : 1) quantize_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, const float* __restrict__ gs_in,
     const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ gs_out, float* __restrict__ block_err) {
+  __shared__ ScaleTables tab;
   const int64_t nblk = cols / 16;
-  const int64_t total = rows * nblk;
   const int64_t atoms_per_group = (nblk + 3) / 4;
   const float sg = global_scale(gs_in, amax_bits);
   if (gs_out && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = sg;
   const float d6 = __fmul_rn(6.0f, sg);
+  if (threadIdx.x < 128) {
+    const float eff = __fmul_rn(e4m3_to_float(threadIdx.x), sg);
+    tab.eff[threadIdx.x] = eff;
+    tab.rcp[threadIdx.x] = eff == 0.0f ? 0.0f : __frcp_rn(eff);
+  }
+  __syncthreads();
 
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const bool small = total < (int64_t(1) << 32);
-  // When a row's block count is a multiple of 4, four consecutive blocks (lanes
-  // 4j..4j+3) own four consecutive bytes of the swizzled scale layout.
-  const bool pack_scales = SWZ && (nblk & 3) == 0;
+  const int64_t chunks = (nblk + 31) / 32;  // warp tasks per row
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+  int64_t r0, r_step, c0, c_step;
+  if (nwarps >= chunks) {
+    r_step = nwarps / chunks;
+    r0 = w / chunks;
+    c0 = w % chunks;
+    c_step = chunks;
+    if (r0 >= r_step) return;  // the few warps past the last whole set of chunks
+  } else {
+    r0 = 0;
+    r_step = 1;
+    c0 = w;
+    c_step = nwarps;
+  }
   const int lane = threadIdx.x & 31;
-  // warp-uniform loop: every lane of a warp runs the same iterations
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31); base < total;
-       base += stride) {
-    const int64_t b = base + lane;
-    const bool active = b < total;
-    int64_t r = 0, cb = 0;
-    uint32_t best_s = 0;
-    if (active) {
-    if (small) {
-      const uint32_t b32 = static_cast<uint32_t>(b), n32 = static_cast<uint32_t>(nblk);
-      const uint32_t r32 = b32 / n32;
-      r = r32;
-      cb = b32 - r32 * n32;
-    } else {
-      r = b / nblk;
-      cb = b - r * nblk;
-    }
-    const uint16_t* src = x + r * ld + cb * 16;
-    const uint4 lo = ld_nc_v4(src), hi = ld_nc_v4(src + 8);
-    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-    uint64_t x2[8];  // the block as signed binary32 pairs (BF16 widening is exact)
-    uint32_t mb = 0;
+  for (int64_t r = r0; r < rows; r += r_step) {
+    const uint16_t* xrow = x + r * ld;
+    uint8_t* crow = codes + r * (cols / 2);
+    const int64_t sf_row = SWZ ? (r >> 7) * atoms_per_group * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 : r * nblk;
+    for (int64_t c = c0; c < chunks; c += c_step) {
+      const int64_t cb = c * 32 + lane;
+      const bool active = cb < nblk;
+      uint32_t best_s = 0;
+      if (active) {
+        const uint4 lo = ld_nc_v4(xrow + cb * 16), hi = ld_nc_v4(xrow + cb * 16 + 8);
+        const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        uint64_t x2[8];  // the block as signed binary32 pairs (BF16 widening is exact)
+        uint32_t mb = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      x2[i] = pack2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-      mb = __vmaxu2(mb, w[i] & 0x7FFF7FFFu);
-    }
-    const float amax_b = bf16_bits_to_float(max(mb & 0xFFFFu, mb >> 16));
-    const float vb = __fdiv_rn(amax_b, d6);
+        for (int i = 0; i < 8; ++i) {
+          x2[i] = pack2(__uint_as_float(wd[i] << 16), __uint_as_float(wd[i] & 0xFFFF0000u));
+          mb = __vmaxu2(mb, wd[i] & 0x7FFF7FFFu);
+        }
+        const float amax_b = bf16_bits_to_float(max(mb & 0xFFFFu, mb >> 16));
+        const float vb = __fdiv_rn(amax_b, d6);
 
-    // candidate f = 1: the absmax scale
-    best_s = cvt_e4m3_satfinite(vb);
-    float best_eff = __fmul_rn(e4m3_to_float(best_s), sg);
-    uint32_t best_c0, best_c1;
-    encode_codes(x2, best_eff, best_c0, best_c1);
-    float best_e = 0.0f;
-    if (MODE == 1 || block_err) best_e = block_sse(x2, best_c0, best_c1, best_eff);
+        // candidate f = 1: the absmax scale
+        best_s = cvt_e4m3_satfinite(vb);
+        const float best_eff = tab.eff[best_s];
+        uint32_t best_c0, best_c1;
+        encode_codes(x2, best_eff, tab.rcp[best_s], best_c0, best_c1);
+        float best_e = 0.0f;
+        if (MODE == 1 || block_err) best_e = block_sse(x2, best_c0, best_c1, best_eff);
 
-    if (MODE == 1) {
-      const float factors[7] = {0.9f, 0.8f, 0.7f, 0.6f, 0.5f, 0.4f, 0.3f};
-      uint32_t prev_s = best_s;
+        if (MODE == 1) {
+          const float factors[7] = {0.9f, 0.8f, 0.7f, 0.6f, 0.5f, 0.4f, 0.3f};
+          uint32_t prev_s = best_s;
 #pragma unroll 1
-      for (int i = 0; i < 7; ++i) {
-        const uint32_t s = cvt_e4m3_satfinite(__fmul_rn(factors[i], vb));
-        if (s == prev_s) continue;  // same scale, same error: never a strict improvement
-        prev_s = s;
-        const float eff = __fmul_rn(e4m3_to_float(s), sg);
-        // Clip bound: if the block maximum lands above the 4|6 midpoint it is coded
-        // as 6, and its term alone makes e >= RN(d*d) with d = fma(-6, eff, amax_b):
-        // each fma of the error sum adds a non-negative term to a non-negative sum,
-        // and rounding is monotone.  Such a candidate cannot strictly improve when
-        // RN(d*d) >= best_e.  When d >= 0 (the maximum is clipped) later candidates,
-        // with smaller eff, have a larger d and cannot either, so the walk stops.
-        if (eff != 0.0f && __fmul_rn(amax_b, __frcp_rn(eff)) > 5.0f) {
-          const float d = __fmaf_rn(-6.0f, eff, amax_b);
-          if (__fmul_rn(d, d) >= best_e) {
-            if (d >= 0.0f) break;
-            continue;
+          for (int i = 0; i < 7; ++i) {
+            const uint32_t s = cvt_e4m3_satfinite(__fmul_rn(factors[i], vb));
+            if (s == prev_s) continue;  // same scale, same error: never a strict improvement
+            prev_s = s;
+            const float eff = tab.eff[s], rcp = tab.rcp[s];
+            // Clip bound: if the block maximum lands above the 4|6 midpoint it is coded
+            // as 6, and its term alone makes e >= RN(d*d) with d = fma(-6, eff, amax_b):
+            // each fma of the error sum adds a non-negative term to a non-negative sum,
+            // and rounding is monotone.  Such a candidate cannot strictly improve when
+            // RN(d*d) >= best_e.  When d >= 0 (the maximum is clipped) later candidates,
+            // with smaller eff, have a larger d and cannot either, so the walk stops.
+            if (eff != 0.0f && __fmul_rn(amax_b, rcp) > 5.0f) {
+              const float d = __fmaf_rn(-6.0f, eff, amax_b);
+              if (__fmul_rn(d, d) >= best_e) {
+                if (d >= 0.0f) break;
+                continue;
+              }
+            }
+            uint32_t c0w, c1w;
+            encode_codes(x2, eff, rcp, c0w, c1w);
+            const float e = block_sse(x2, c0w, c1w, eff);
+            if (e < best_e) {
+              best_e = e;
+              best_s = s;
+              best_c0 = c0w;
+              best_c1 = c1w;
+            }
           }
         }
-        uint32_t c0, c1;
-        encode_codes(x2, eff, c0, c1);
-        const float e = block_sse(x2, c0, c1, eff);
-        if (e < best_e) {
-          best_e = e;
-          best_s = s;
-          best_c0 = c0;
-          best_c1 = c1;
-        }
+        *reinterpret_cast<uint2*>(crow + cb * 8) = make_uint2(best_c0, best_c1);
+        if (!SWZ) scales[sf_row + cb] = static_cast<uint8_t>(best_s);
+        if (block_err) block_err[r * nblk + cb] = best_e;
       }
-    }
-
-    *reinterpret_cast<uint2*>(codes + r * (cols / 2) + cb * 8) = make_uint2(best_c0, best_c1);
-    if (!pack_scales) {
-      if (SWZ)
-        scales[swizzled_offset(r, cb, atoms_per_group)] = static_cast<uint8_t>(best_s);
-      else
-        scales[b] = static_cast<uint8_t>(best_s);
-    }
-    if (block_err) block_err[b] = best_e;
-    }  // active
-    if (pack_scales) {
-      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, best_s, 1);
-      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, best_s, 2);
-      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, best_s, 3);
-      if (active && (cb & 3) == 0)
-        *reinterpret_cast<uint32_t*>(scales + swizzled_offset(r, cb, atoms_per_group)) =
-            best_s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      if (SWZ) {
+        // lanes 4j..4j+3 hold four consecutive blocks of the row: one 32-bit store of
+        // their scale bytes (a lane past the row end contributes the padding's 0)
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, best_s, 1);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, best_s, 2);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, best_s, 3);
+        if (active && (lane & 3) == 0)
+          *reinterpret_cast<uint32_t*>(scales + sf_row + (cb >> 2) * 512) =
+              best_s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      }
     }
   }
 }
