@@ -276,6 +276,15 @@ def work_units(cfg):
     return flops, elems
 
 
+def gemm_kernel_name(M: int, N: int) -> str:
+    """The kernel the library picks for an M x N output (its launch dispatch)."""
+    if M <= 32:
+        return "gemm_decode_kernel (tcgen05 mxf4nvf4, split-K)"
+    if M > 128 and N > 128:
+        return "gemm_pair_kernel (tcgen05 cta_group::2 mxf4nvf4)"
+    return "gemm_kernel (tcgen05 mxf4nvf4)"
+
+
 def run_ours(args, rank, world, local):
     import torch
     import w4a4_gemm_quantize_b200 as nv
@@ -325,7 +334,7 @@ def run_ours(args, rank, world, local):
     traffic = profiled_traffic("gemm", args.workload)
     roofline = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                 "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4), "traffic": traffic,
-                "kernel": "gemm_kernel (tcgen05 mxf4nvf4), launch gemm_1 (M x N1 x K1)",
+                "kernel": f"{gemm_kernel_name(cfg['M'], cfg['N1'])}, launch gemm_1 (M x N1 x K1)",
                 "peak_source": f"{peaks['source']} bf16 {'sustained' if long_region else 'burst'} x {FP4_PER_BF16:g}"}
     comps = {}
     for n in names:
@@ -334,7 +343,10 @@ def run_ours(args, rank, world, local):
             t = 2 * M * N * K / (per_group[n] * 1e-3) / 1e12
             comps[n] = {"us": round(per_group[n] * 1e3, 1), "TFLOP/s": round(t, 1), "frac_fp4_peak": round(t / fp4_peak, 4)}
         else:
-            bpe = 2.5625  # read 2 B of BF16, write 0.5 B of codes + 1/16 B of scales per element
+            # quantize (two-pass, the per-tensor scale computed in the step): 2 B read by
+            # the amax pass + 2 B read and 0.5625 B written by the encode pass; dequantize:
+            # 0.5625 B read + 2 B written
+            bpe = 2.5625 if n.startswith("dequantize") else 4.5625
             gbs = elems[n] * bpe / (per_group[n] * 1e-3) / 1e9
             comps[n] = {"us": round(per_group[n] * 1e3, 1), "GB/s": round(gbs, 1),
                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_elem": bpe}
