@@ -318,13 +318,21 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 // the MMAs).  Three sets rotate over K-tiles so that one set's barrier round trip
 // overlaps the others' copies.  The leader's set also waits for the stage's A/B
 // bytes before it arrives, so the MMA issuer waits on one barrier per K-tile: every
-// wait in the issuing thread lets the tensor pipe's queue run dry, and with four
-// MMAs per wait that costs a tenth of the pipe's time per extra wait.  A stage's region is free again when its
-// shared-memory slot is: the producer reloads stage s only after the MMAs that
-// read it completed, so no separate release barrier is needed.
+// wait in the issuing thread lets the tensor pipe's queue run dry (with four MMAs
+// per wait the pipe already runs at about 85 % of its rate).  The peer's set
+// gathers its four warps on a local barrier and one of them arrives with a
+// cluster-scope release, which orders the set's TMEM stores before the leader's MMA
+// reads them (one remote release per K-tile: four of them cost ~10 % of the GEMM).
+// Scale factors have their own producer and shared-memory slots, refilled as soon
+// as a set has read them, so they land several K-tiles ahead of their MMAs.  A stage's region is free again when its shared-memory
+// slot is: the producer reloads stage s only after the MMAs that read it
+// completed, so no separate release barrier is needed.  Each K-tile's MMAs end with
+// one commit that arrives on both CTAs' `empty` barriers.
 //
-// Epilogue: 8 warps (2 per sub-partition) read the accumulator, release it, and
-// write BF16 through 128-byte-swizzled shared-memory boxes with TMA stores.
+// Epilogue: 8 warps (2 per sub-partition) read the accumulator, release it (the
+// peer's warps with a relaxed arrive: they have only read TMEM, and waited for the
+// reads), and write BF16 through 128-byte-swizzled shared-memory boxes with TMA
+// stores.
 
 struct PairCfg {
   static constexpr int BM = 128;                      // rows of A per CTA (256 per pair)
@@ -346,7 +354,8 @@ struct PairCfg {
   static constexpr int MMA_WARP = EPI_WARPS + 1;      // 9
   static constexpr int SF_WARP0 = EPI_WARPS + 2;      // 10..
   static constexpr int SF_SETS = 3;                   // sets of 4 scale warps, rotating over K-tiles
-  static constexpr int THREADS = (EPI_WARPS + 2 + 4 * SF_SETS) * 32;
+  static constexpr int SF_PRODUCER_WARP = SF_WARP0 + 4 * SF_SETS;  // 22
+  static constexpr int THREADS = (SF_PRODUCER_WARP + 1) * 32;
   static constexpr int GROUP_M = 8;                   // in 256-row tiles
   static constexpr int SF_REGIONS = STAGES;           // one TMEM scale region per pipeline stage
   static constexpr int SF_COLS = 48;                  // A: 16 columns, B: 32 columns per K-tile
@@ -374,8 +383,10 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sC + Cfg::C_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* sf_full = empty + STAGES;
-  uint64_t* sf_ready = sf_full + STAGES;
-  uint64_t* acc_full = sf_ready + R;
+  uint64_t* sf_empty = sf_full + STAGES;
+  uint64_t* sf_ready = sf_empty + STAGES;
+  uint64_t* set_done = sf_ready + STAGES;  // [SF_SETS]: the four warps of a set (peer CTA)
+  uint64_t* acc_full = set_done + Cfg::SF_SETS;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -396,8 +407,10 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sf_full[s], 1);
+      mbar_init(&sf_empty[s], 4);  // the four warps of the set that read the slot
     }
-    for (int r = 0; r < R; ++r) mbar_init(&sf_ready[r], 8);  // 4 scale warps in each CTA of the pair
+    for (int r = 0; r < R; ++r) mbar_init(&sf_ready[r], 5);  // 4 leader warps + 1 arrival from the peer
+    for (int q = 0; q < Cfg::SF_SETS; ++q) mbar_init(&set_done[q], 4);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * Cfg::EPI_WARPS);
     mbar_init(drain, 1);
@@ -440,14 +453,11 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             break;
           }
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (Cfg::A_BYTES + Cfg::B_BYTES));
-          mbar_arrive_expect_tx(&sf_full[s], Cfg::SFA_BYTES + Cfg::SFB_BYTES);
           const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0u);
           tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tmap_a, bar, kt * Cfg::KTILE_BYTES,
                            tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM);
           tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tmap_b, bar, kt * Cfg::KTILE_BYTES,
                            tn * Cfg::BN + static_cast<int>(rank) * 128);
-          tma_load_3d(sSFA + s * Cfg::SFA_BYTES, &tmap_sfa, &sf_full[s], 0, kt * 4, tm * 2 + static_cast<int>(rank));
-          tma_load_3d(sSFB + s * Cfg::SFB_BYTES, &tmap_sfb, &sf_full[s], 0, kt * 4, tn * 2);
           issued_last[s] = kc;
         }
       }
@@ -455,7 +465,6 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         for (int s = 0; s < STAGES; ++s)
           if (issued_last[s] >= 0) {
             const uint32_t par = static_cast<uint32_t>(issued_last[s] / STAGES) & 1u;
-            mbar_wait_drain(&sf_full[s], par, status);
             if (rank == 0) mbar_wait_drain(&full[s], par, status);
           }
       }
@@ -503,26 +512,63 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         mbar_wait_drain(drain, 0u, status);
       }
     }
+  } else if (warp == Cfg::SF_PRODUCER_WARP) {
+    if (lane == 0) {
+      // ---------------- scale-factor producer (both CTAs) ----------------
+      // Slot s is refilled as soon as the set that copied K-tile kc-5 has read it,
+      // several K-tiles before the MMAs reach kc, so the scale copy is not on the
+      // critical path of a stage's reload.
+      int issued_last[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
+      int kc = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs) {
+        int tm, tn;
+        tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
+        for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+          const int s = kc % STAGES;
+          if (kc >= STAGES && !mbar_wait(&sf_empty[s], (static_cast<uint32_t>(kc / STAGES) & 1u) ^ 1u, abort_flag,
+                                         status, kErrWaitEmpty + 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sf_full[s], Cfg::SFA_BYTES + Cfg::SFB_BYTES);
+          tma_load_3d(sSFA + s * Cfg::SFA_BYTES, &tmap_sfa, &sf_full[s], 0, kt * 4, tm * 2 + static_cast<int>(rank));
+          tma_load_3d(sSFB + s * Cfg::SFB_BYTES, &tmap_sfb, &sf_full[s], 0, kt * 4, tn * 2);
+          issued_last[s] = kc;
+        }
+      }
+      if (*abort_flag)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_last[s] >= 0)
+            mbar_wait_drain(&sf_full[s], static_cast<uint32_t>(issued_last[s] / STAGES) & 1u, status);
+    }
   } else if (warp >= Cfg::SF_WARP0) {
     // ---------------- scale warps (both CTAs): shared memory -> TMEM ----------------
     const uint32_t quarter = static_cast<uint32_t>(warp & 3);
     const int set = (warp - Cfg::SF_WARP0) >> 2;
     const uint32_t sf_ready_leader0 = mapa_shared(smem_u32(&sf_ready[0]), 0u);
-    int kc = 0;
+    int kc = 0, handled = 0;
     bool ok = true;
     for (int t = pair; t < num_tiles && ok; t += npairs) {
       for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
         if (kc % Cfg::SF_SETS != set) continue;
         const int s = kc % STAGES;
         const int r = s;
-        // the stage's scales have landed; the producer reloaded this stage only after
-        // the MMAs that last read region r had completed
-        if (!warp_wait_cluster(&sf_full[s], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
-                               kErrWaitFull + 2)) {
+        const uint32_t prev = (static_cast<uint32_t>(kc / STAGES) & 1u) ^ 1u;  // parity of K-tile kc-5's phase
+        // A parity wait is only sound when the barrier is at most one phase behind, and
+        // the sets rotate: first see K-tile kc-5 through slot s (its set has read the
+        // slot, so those scales had landed), then wait for kc's scales.
+        if (kc >= STAGES &&
+            !warp_wait(&sf_empty[s], prev, abort_flag, status, kErrWaitFull + 3)) {
           ok = false;
           break;
         }
-        tc_fence_after();
+        if (!warp_wait(&sf_full[s], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status, kErrWaitFull + 2)) {
+          ok = false;
+          break;
+        }
         const uint8_t* fa = sSFA + s * Cfg::SFA_BYTES + lane * 16;
         const uint8_t* fb = sSFB + s * Cfg::SFB_BYTES + lane * 16;
         uint32_t va[16], vb[32];
@@ -542,6 +588,14 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             vb[8 * j + 4 * g + 3] = b4.w;
           }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_empty[s]);  // the slot may be refilled
+        // TMEM region r is free once the MMAs of K-tile kc-5 have completed
+        if (kc >= STAGES && !warp_wait_cluster(&empty[s], prev, abort_flag, status, kErrWaitFull + 4)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         const uint32_t t_sf = tmem_base + (quarter * 32u << 16) + Cfg::TMEM_SF + r * Cfg::SF_COLS;
         tmem_st_32x32b_x16(t_sf, va);
         tmem_st_32x32b_x32(t_sf + 16, vb);
@@ -553,12 +607,20 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          if (rank == 0)
-            mbar_arrive(&sf_ready[r]);
-          else
-            mbar_arrive_cluster_relaxed(sf_ready_leader0 + r * 8u);
+        if (rank == 0) {
+          if (lane == 0) mbar_arrive(&sf_ready[r]);
+        } else {
+          if (lane == 0) mbar_arrive(&set_done[set]);
+          if (quarter == static_cast<uint32_t>(set & 3)) {  // one warp of the set
+            const uint32_t hand = static_cast<uint32_t>(handled & 1);
+            if (!warp_wait(&set_done[set], hand, abort_flag, status, kErrWaitFull + 5)) {
+              ok = false;
+              break;
+            }
+            if (lane == 0) mbar_arrive_cluster(sf_ready_leader0 + r * 8u);
+          }
         }
+        ++handled;
       }
     }
   } else {
@@ -635,18 +697,30 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------------------------
-// Decode kernel (M <= 32): weights on the 128-row side of the MMA, split-K
+// Decode kernel (M <= 32): weights on the 128-row side of the MMA, stream-K
 // ---------------------------------------------------------------------------------------------
 //
 // For a handful of activation rows the GEMM is a stream over the weights, so the
 // weight matrix B takes the MMA's 128-row A slot (D^T = B A^T, 128 x 32 x 64 per
-// instruction) and each CTA handles one 128-row weight tile over a slice of K.
-// Partial FP32 tiles go to the workspace; the last CTA of a weight tile (by an
-// atomic counter) sums the slices in slice order, applies s_gA s_gB and writes
-// C (transposed back) in BF16, so the result does not depend on arrival order.
+// instruction).  The stream is split evenly over the CTAs (one per SM): the K-tiles
+// of all 128-row weight tiles form one sequence of units, tile-major, and CTA c
+// takes units [c U / G, (c+1) U / G).  Every SM therefore streams the same number
+// of weight bytes, whatever the number of tiles.  A CTA's range can cross tile
+// boundaries; its part of one tile is a "segment" with its own accumulator, and
+// TMEM holds two accumulators so that the MMAs of a segment overlap the epilogue
+// of the one before.  A segment that covers a whole tile writes C.  Otherwise it
+// stores its FP32 partial tile; the segment of the tile that finishes last (atomic
+// counter) sums the tile's partials in segment order -- the result does not
+// depend on arrival order -- applies s_gA s_gB and writes C (transposed back) in
+// BF16, then clears the counter for the next call.
+//
+// Scale factors reach TMEM through four "scale warps" (tcgen05.st of each lane's
+// 16-byte atom lines into a per-stage region, as in the pair kernel), not through
+// tcgen05.cp: two copies per 128 x 32 x 64 MMA made the in-order tensor pipe, not
+// HBM, the limit.  The MMA issuer waits on one barrier per K-tile.
 
 struct DecodeCfg {
-  static constexpr int BM = 128;                 // weight rows per CTA
+  static constexpr int BM = 128;                 // weight rows per tile
   static constexpr int BN = 32;                  // activation rows (padded)
   static constexpr int KTILE_BYTES = 128;
   static constexpr int A_BYTES = BM * KTILE_BYTES;   // 16 KB of weight codes
@@ -655,18 +729,40 @@ struct DecodeCfg {
   static constexpr int SFA_BYTES = 4 * SF_ATOM;
   static constexpr int SFB_BYTES = 4 * SF_ATOM;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = 4;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
-  static constexpr int THREADS = 192;            // warps 0-3 epilogue, 4 producer, 5 MMA
-  static constexpr int TMEM_SF = 32;             // two scale regions of 32 columns after the accumulator
-  static constexpr int TMEM_COLS = 128;
+  static constexpr int STAGES = 8;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
+  static constexpr int THREADS = 320;            // warps 0-3 epilogue, 4 producer, 5 MMA, 6-9 scales
+  static constexpr int SF_WARP0 = 6;
+  static constexpr int TMEM_ACC = 0;             // two accumulators of 32 columns
+  static constexpr int TMEM_SF = 64;             // one scale region of 32 columns per stage
+  static constexpr int TMEM_COLS = 512;
+  static_assert(TMEM_SF + STAGES * 32 <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
+
+// Largest decode grid (SM count) the workspace query provisions partial-tile slots for.
+constexpr int kMaxDecodeGrid = 296;
+
+// The CTA whose unit range [c U / G, (c+1) U / G) holds unit u.
+__host__ __device__ inline int64_t decode_cta_of_unit(int64_t u, int64_t U, int64_t G) {
+  int64_t c = u * G / U;  // floor(c U / G) <= u for this c
+  while (c + 1 < G && (c + 1) * U / G <= u) ++c;
+  return c;
+}
+
+// Segments a tile of KT units can be cut into when every CTA holds at least
+// U / G units (the partial-tile slots per tile in the workspace).
+__host__ __device__ inline int64_t decode_max_segments(int64_t KT, int64_t U, int64_t G) {
+  const int64_t per = U / G < 1 ? 1 : U / G;
+  const int64_t s = (KT - 1) / per + 2;
+  return s < KT ? s : KT;
+}
 
 __global__ void __launch_bounds__(DecodeCfg::THREADS)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                        const uint8_t* __restrict__ sf_w, const uint8_t* __restrict__ sf_x,
                        const float* __restrict__ a_gs, const float* __restrict__ b_gs, uint16_t* __restrict__ C,
-                       int M, int N, int K, int64_t ldc, int splits, float* __restrict__ partial,
+                       int M, int N, int K, int64_t ldc, int max_seg, float* __restrict__ partial,
                        uint32_t* __restrict__ counters, uint32_t* __restrict__ status) {
   using Cfg = DecodeCfg;
   constexpr int STAGES = Cfg::STAGES;
@@ -678,25 +774,33 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
   uint8_t* sSFB = sSFA + STAGES * Cfg::SFA_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * Cfg::SFB_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint64_t* drain = acc_full + 1;
+  uint64_t* sf_ready = empty + STAGES;
+  uint64_t* acc_full = sf_ready + STAGES;  // [2]
+  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  volatile uint32_t* last_flag = tmem_slot + 2;
+  volatile uint32_t* decision = tmem_slot + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x / splits, split = blockIdx.x - tile * splits;
   const int k_atoms = (K + 63) / 64;
-  const int k_tiles = (k_atoms + 3) / 4;
-  const int kt0 = static_cast<int>(static_cast<int64_t>(split) * k_tiles / splits);
-  const int kt1 = static_cast<int>(static_cast<int64_t>(split + 1) * k_tiles / splits);
+  const int64_t KT = (k_atoms + 3) / 4;
+  const int64_t T = (N + Cfg::BM - 1) / Cfg::BM;
+  const int64_t U = T * KT;
+  const int64_t G = gridDim.x;
+  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * U / G;
+  const int64_t u1 = (static_cast<int64_t>(blockIdx.x) + 1) * U / G;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 4);  // lane 0 of each scale warp
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);  // lane 0 of each epilogue warp
+    }
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_mbarrier_init();
@@ -716,13 +820,15 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
 
   if (warp == 4) {
     if (lane == 0) {
-      int issued_last[STAGES];
+      // ---------------- producer ----------------
+      int64_t issued_last[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
-      for (int kt = kt0, i = 0; kt < kt1; ++kt, ++i) {
-        const int s = i % STAGES;
+      for (int64_t u = u0, i = 0; u < u1; ++u, ++i) {
+        const int s = static_cast<int>(i % STAGES);
         if (!mbar_wait(&empty[s], (static_cast<uint32_t>(i / STAGES) & 1u) ^ 1u, abort_flag, status, kErrWaitEmpty))
           break;
+        const int tile = static_cast<int>(u / KT), kt = static_cast<int>(u - tile * KT);
         const int ka0 = kt * 4;
         const int na = min(4, k_atoms - ka0);
         const uint32_t sf_bytes = static_cast<uint32_t>(na) * Cfg::SF_ATOM;
@@ -741,11 +847,26 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
     }
   } else if (warp == 5) {
     if (lane == 0) {
+      // ---------------- MMA issuer ----------------
       const uint32_t idesc = idesc_mxf4nvf4(Cfg::BM, Cfg::BN);
       bool ok = true;
-      for (int kt = kt0, i = 0; kt < kt1; ++kt, ++i) {
-        const int s = i % STAGES;
-        if (!mbar_wait(&full[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull)) {
+      int q = 0;  // segment counter of this CTA
+      for (int64_t u = u0, i = 0; u < u1 && ok; ++u, ++i) {
+        const int tile = static_cast<int>(u / KT), kt = static_cast<int>(u - tile * KT);
+        const bool seg_first = (u == u0) || kt == 0;
+        const bool seg_last = (u + 1 == u1) || kt + 1 == KT;
+        const int buf = q & 1;
+        if (seg_first && q >= 2) {
+          if (!mbar_wait(&acc_empty[buf], static_cast<uint32_t>((q >> 1) - 1) & 1u, abort_flag, status,
+                         kErrWaitAccEmpty)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const int s = static_cast<int>(i % STAGES);
+        // the scale warps arrive only after the stage's bytes landed and its scales are in TMEM
+        if (!mbar_wait(&sf_ready[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull)) {
           ok = false;
           break;
         }
@@ -753,68 +874,116 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
         const int na = min(4, k_atoms - kt * 4);
         const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
         const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
-        const uint32_t sfa_base = smem_u32(sSFA + s * Cfg::SFA_BYTES);
-        const uint32_t sfb_base = smem_u32(sSFB + s * Cfg::SFB_BYTES);
-        const uint32_t t_sf = tmem_base + Cfg::TMEM_SF + (i & 1) * 32;
-        for (int j = 0; j < na; ++j) {
-          tc_cp_sf(t_sf + 4 * j, sdesc_sf_tile(sfa_base + j * Cfg::SF_ATOM));
-          tc_cp_sf(t_sf + 16 + 4 * j, sdesc_sf_tile(sfb_base + j * Cfg::SF_ATOM));
-          mma_mxf4nvf4(tmem_base, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
-                       t_sf + 4 * j, t_sf + 16 + 4 * j, (i | j) != 0 ? 1u : 0u);
-        }
+        const uint32_t t_sf = tmem_base + Cfg::TMEM_SF + static_cast<uint32_t>(s) * 32;
+        const uint32_t t_acc = tmem_base + Cfg::TMEM_ACC + buf * Cfg::BN;
+        for (int j = 0; j < na; ++j)
+          mma_mxf4nvf4(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
+                       t_sf + 4 * j, t_sf + 16 + 4 * j, (!seg_first || j != 0) ? 1u : 0u);
         tc_commit(&empty[s]);
+        if (seg_last) {
+          tc_commit(&acc_full[buf]);
+          ++q;
+        }
       }
-      if (ok) {
-        tc_commit(acc_full);
-      } else {
+      if (!ok) {
         tc_commit(drain);
         mbar_wait_drain(drain, 0u, status);
       }
     }
-  } else {
-    // epilogue: lane = weight row n of the tile, 32 columns = activation rows m
-    const int n = tile * Cfg::BM + warp * 32 + lane;
-    warp_wait(acc_full, 0u, abort_flag, status, kErrWaitAccFull);
-    // one decision for all four warps (they meet at the named barrier below)
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (threadIdx.x == 0) *last_flag = *abort_flag ? 0u : 2u;
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    const bool have = *last_flag == 2u;
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    uint32_t v[32];
-    if (have) {
+  } else if (warp >= Cfg::SF_WARP0) {
+    // ---------------- scale warps: shared memory -> TMEM region of the stage ----------------
+    // Each lane writes its 16-byte line of every atom to the four columns the MMA reads
+    // for its 32-lane sub-partition (the 4-way replication of the scale layout).  The
+    // region of stage s is free once the stage's bytes land again: the producer
+    // reloads a stage only after the MMAs that read it have completed.
+    const uint32_t quarter = static_cast<uint32_t>(warp & 3);
+    for (int64_t u = u0, i = 0; u < u1; ++u, ++i) {
+      const int s = static_cast<int>(i % STAGES);
+      if (!warp_wait(&full[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull + 2)) break;
       tc_fence_after();
-      tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16), v);
-      tmem_ld_wait();
-    }
-    const float alpha = __fmul_rn(*a_gs, *b_gs);
-    if (have && splits == 1) {
-      if (n < N)
-        for (int m = 0; m < M; ++m)
-          C[static_cast<int64_t>(m) * ldc + n] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__uint_as_float(v[m]), alpha)));
-    } else if (have) {
-      // this slice's partial tile, then the last slice to finish reduces all of them
-      float4* dst = reinterpret_cast<float4*>(partial + ((static_cast<int64_t>(split) * N + n) * Cfg::BN));
-      if (n < N)
+      const uint8_t* fa = sSFA + s * Cfg::SFA_BYTES + lane * 16;
+      const uint8_t* fb = sSFB + s * Cfg::SFB_BYTES + lane * 16;
+      uint32_t v[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+      for (int j = 0; j < 4; ++j) {
+        const uint4 a4 = *reinterpret_cast<const uint4*>(fa + j * Cfg::SF_ATOM);
+        const uint4 b4 = *reinterpret_cast<const uint4*>(fb + j * Cfg::SF_ATOM);
+        v[4 * j] = a4.x;
+        v[4 * j + 1] = a4.y;
+        v[4 * j + 2] = a4.z;
+        v[4 * j + 3] = a4.w;
+        v[16 + 4 * j] = b4.x;
+        v[16 + 4 * j + 1] = b4.y;
+        v[16 + 4 * j + 2] = b4.z;
+        v[16 + 4 * j + 3] = b4.w;
+      }
+      tmem_st_32x32b_x32(tmem_base + (quarter * 32u << 16) + Cfg::TMEM_SF + static_cast<uint32_t>(s) * 32, v);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sf_ready[s]);
+    }
+  } else {
+    // ---------------- epilogue (warps 0-3): lane = weight row n, 32 columns = activation rows m ----------------
+    const float alpha = __fmul_rn(*a_gs, *b_gs);
+    int q = 0;
+    for (int64_t u = u0; u < u1; ++q) {
+      const int tile = static_cast<int>(u / KT);
+      const int64_t tile_end = (static_cast<int64_t>(tile) + 1) * KT;
+      const int64_t seg_end = tile_end < u1 ? tile_end : u1;  // this segment: units [u, seg_end)
+      const bool whole = (u == static_cast<int64_t>(tile) * KT) && seg_end == tile_end;
+      const int buf = q & 1;
+      const bool got = warp_wait(&acc_full[buf], static_cast<uint32_t>(q >> 1) & 1u, abort_flag, status,
+                                 kErrWaitAccFull);
+      uint32_t v[32];
+      if (got) {
+        tc_fence_after();
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + Cfg::TMEM_ACC + buf * Cfg::BN, v);
+        tmem_ld_wait();
+        tc_fence_before();
+      }
+      __syncwarp();
+      if (got && lane == 0) mbar_arrive(&acc_empty[buf]);
+      // one decision for the four warps: go on only if none of them gave up
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 0) *decision = *abort_flag ? 0u : 1u;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const bool go = *decision == 1u;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!go) break;
+      const int n = tile * Cfg::BM + warp * 32 + lane;
+      if (whole) {
+        if (n < N)
+          for (int m = 0; m < M; ++m)
+            C[static_cast<int64_t>(m) * ldc + n] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__uint_as_float(v[m]), alpha)));
+      } else {
+        const int64_t c_first = decode_cta_of_unit(static_cast<int64_t>(tile) * KT, U, G);
+        const int64_t c_last = decode_cta_of_unit(tile_end - 1, U, G);
+        const int seg = static_cast<int>(blockIdx.x - c_first);
+        const int nseg = static_cast<int>(c_last - c_first + 1);
+        float* slot = partial + ((static_cast<int64_t>(tile) * max_seg + seg) * Cfg::BM + warp * 32 + lane) * Cfg::BN;
+        float4* dst = reinterpret_cast<float4*>(slot);
+        const int mq = (M + 3) / 4;  // only the activation rows that exist are kept
+        for (int i = 0; i < mq; ++i)
           dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
                                __uint_as_float(v[4 * i + 3]));
-      __threadfence();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (threadIdx.x == 0) *last_flag = (atomicAdd(&counters[tile], 1u) == static_cast<uint32_t>(splits - 1)) ? 1u : 0u;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (*last_flag) {
-        __threadfence();
-        if (n < N) {
+        // the four warps' partial rows are ordered before thread 0's release by the
+        // barrier; the segment that arrives last acquires every other segment's rows
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (threadIdx.x == 0)
+          *decision = (atom_add_acq_rel_gpu(&counters[tile], 1u) == static_cast<uint32_t>(nseg - 1)) ? 2u : 1u;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const bool last = *decision == 2u;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (last) {
           float acc[32];
 #pragma unroll
           for (int m = 0; m < 32; ++m) acc[m] = 0.0f;
-          for (int sp = 0; sp < splits; ++sp) {
-            const float4* src = reinterpret_cast<const float4*>(partial + ((static_cast<int64_t>(sp) * N + n) * Cfg::BN));
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
+          for (int sg = 0; sg < nseg; ++sg) {
+            const float4* src = reinterpret_cast<const float4*>(
+                partial + ((static_cast<int64_t>(tile) * max_seg + sg) * Cfg::BM + warp * 32 + lane) * Cfg::BN);
+            for (int i = 0; i < mq; ++i) {
               const float4 f = __ldcg(src + i);
               acc[4 * i] = __fadd_rn(acc[4 * i], f.x);
               acc[4 * i + 1] = __fadd_rn(acc[4 * i + 1], f.y);
@@ -822,12 +991,14 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
               acc[4 * i + 3] = __fadd_rn(acc[4 * i + 3], f.w);
             }
           }
-          for (int m = 0; m < M; ++m)
-            C[static_cast<int64_t>(m) * ldc + n] =
-                __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(acc[m], alpha)));
+          if (n < N)
+            for (int m = 0; m < M; ++m)
+              C[static_cast<int64_t>(m) * ldc + n] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(acc[m], alpha)));
+          if (threadIdx.x == 0) counters[tile] = 0u;  // ready for the next call
         }
-        if (threadIdx.x == 0) counters[tile] = 0u;  // ready for the next call
       }
+      u = seg_end;
     }
   }
 
@@ -961,14 +1132,10 @@ cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float
                             static_cast<int>(N), static_cast<int>(K), status);
 }
 
-// Slices of K per 128-row weight tile: as many as fit in one wave of two CTAs per SM.
-int decode_splits(int64_t N, int64_t K, int sms) {
-  const int64_t tiles = (N + 127) / 128;
-  const int64_t k_tiles = (K + 255) / 256;
-  int64_t s = 2 * static_cast<int64_t>(sms) / tiles;
-  if (s > k_tiles / 2) s = k_tiles / 2;
-  if (s > 16) s = 16;
-  return static_cast<int>(s < 1 ? 1 : s);
+// CTAs of the stream-K decode kernel: one per SM, at most one per unit.
+int64_t decode_grid(int64_t N, int64_t K, int sms) {
+  const int64_t U = ((N + DecodeCfg::BM - 1) / DecodeCfg::BM) * ((K + 255) / 256);
+  return U < sms ? U : sms;
 }
 
 cudaError_t launch_decode(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
@@ -987,16 +1154,15 @@ cudaError_t launch_decode(const uint8_t* a_codes, const uint8_t* a_sf, const flo
                                     DecodeCfg::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  const int tiles = static_cast<int>((N + 127) / 128);
-  const int splits = decode_splits(N, K, sms);
+  const int64_t KT = (K + 255) / 256;
+  const int64_t U = ((N + DecodeCfg::BM - 1) / DecodeCfg::BM) * KT;
+  const int64_t G = decode_grid(N, K, sms > kMaxDecodeGrid ? kMaxDecodeGrid : sms);
+  const int max_seg = static_cast<int>(decode_max_segments(KT, U, G));
+  // the counters were cleared together with the status word (gemm_zero_bytes)
   uint32_t* counters = reinterpret_cast<uint32_t*>(scratch);
   float* partial = reinterpret_cast<float*>(scratch + decode_counter_bytes(N));
-  if (splits > 1) {
-    cudaError_t e = cudaMemsetAsync(counters, 0, static_cast<size_t>(tiles) * 4, stream);
-    if (e != cudaSuccess) return e;
-  }
-  gemm_decode_kernel<<<tiles * splits, DecodeCfg::THREADS, DecodeCfg::SMEM_BYTES, stream>>>(
-      tw, tx, b_sf, a_sf, a_gs, b_gs, c, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), ldc, splits,
+  gemm_decode_kernel<<<static_cast<unsigned>(G), DecodeCfg::THREADS, DecodeCfg::SMEM_BYTES, stream>>>(
+      tw, tx, b_sf, a_sf, a_gs, b_gs, c, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), ldc, max_seg,
       partial, counters, status);
   return cudaGetLastError();
 }
@@ -1028,8 +1194,17 @@ cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint
 
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
   if (M > DecodeCfg::BN) return 0;
-  const int splits = decode_splits(N, K, 148 * 2);  // upper bound over SM counts up to 296
-  return decode_counter_bytes(N) + static_cast<size_t>(splits) * N * DecodeCfg::BN * 4;
+  // partial-tile slots for the largest grid the launcher uses (more CTAs, more segments)
+  const int64_t KT = (K + 255) / 256;
+  const int64_t T = (N + DecodeCfg::BM - 1) / DecodeCfg::BM;
+  const int64_t G = decode_grid(N, K, kMaxDecodeGrid);
+  const int64_t max_seg = decode_max_segments(KT, T * KT, G);
+  return decode_counter_bytes(N) + static_cast<size_t>(T * max_seg) * DecodeCfg::BM * DecodeCfg::BN * 4;
+}
+
+size_t gemm_zero_bytes(int64_t M, int64_t N, int64_t) {
+  // the status word, and for the decode kernel its tile counters right after the status block
+  return M <= DecodeCfg::BN ? 256 + decode_counter_bytes(N) : sizeof(uint32_t);
 }
 
 cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,

@@ -256,11 +256,18 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// Relaxed arrive on an mbarrier that may live in the other CTA.  For a thread whose
-// only work before the arrive is tensor-memory traffic it has already waited for
-// (tcgen05.wait::st / wait::ld, then tcgen05.fence::before_thread_sync): there are
-// no generic-proxy writes to publish, and a cluster-scope release costs about as much
-// as a K-tile of MMAs.
+// Atomic add with acquire-release semantics at GPU scope; returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
+// Relaxed arrive on an mbarrier that may live in the other CTA, for a thread whose
+// only work before the arrive is tensor-memory loads it has already waited for
+// (tcgen05.wait::ld): it publishes no writes, so nothing needs a release, and a
+// cluster-scope release costs about as much as a K-tile of MMAs.  (Tensor-memory
+// stores that another CTA's MMA will read do need the release.)
 __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
