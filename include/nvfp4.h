@@ -119,8 +119,11 @@ nvfp4_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, nvfp4
                               int64_t ld_out, void *stream);
 
 /* Workspace nvfp4_gemm needs (device memory, any content on entry): 256 bytes
- * for the status word, plus, when M <= 32, room for the split-K partial tiles of
- * the small-M kernel (counters and FP32 partials, about N * 128 * slices bytes). */
+ * for the status word, plus, when M <= 32, the small-M kernel's per-tile counters
+ * and FP32 partial tiles (the weight stream is split evenly over the SMs, so a
+ * 128-row weight tile can be cut into a few K segments: about
+ * N * 128 * segments bytes, a few MB for 8B-class layers).  nvfp4_gemm clears the
+ * status word and the counters itself (one memset on `stream`). */
 size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Block-scaled W4A4 GEMM, C = (A s_a)(B s_b)^T * s_gA * s_gB, FP32 accumulation,
