@@ -179,7 +179,8 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const f
   if (st != NVFP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* status = static_cast<uint32_t*>(workspace);
-  if (cudaMemsetAsync(status, 0, nvfp4::gemm_zero_bytes(M, N, K), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  const size_t zero = nvfp4::gemm_zero_bytes(M, N, K);
+  if (zero > 0 && cudaMemsetAsync(status, 0, zero, s) != cudaSuccess) return NVFP4_ERR_CUDA;
   const cudaError_t e = nvfp4::launch_gemm(a_codes, a_scales, a_global_scale, M, b_codes, b_scales, b_global_scale,
                                            N, K, static_cast<uint16_t*>(c), ldc, status, s);
   if (e == cudaErrorInvalidValue) return NVFP4_ERR_CUDA;

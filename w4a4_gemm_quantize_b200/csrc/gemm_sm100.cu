@@ -149,6 +149,11 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The set-up above overlaps the previous kernel's tail (programmatic launch);
+  // from here on the operands it wrote are visible.  The status word is cleared
+  // here, long before any bounded wait could give up.
+  grid_dependency_wait();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
 
   if (warp == Cfg::PRODUCER_WARP) {
     if (lane == 0) {
@@ -433,6 +438,9 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // set-up overlapped the previous kernel's tail; its outputs are visible from here
+  grid_dependency_wait();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
 
   if (warp == Cfg::PRODUCER_WARP) {
     if (lane == 0) {
@@ -817,6 +825,9 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // set-up overlapped the previous kernel's tail; its outputs are visible from here
+  // (the status word and tile counters were cleared by the memset launched before)
+  grid_dependency_wait();
 
   if (warp == 4) {
     if (lane == 0) {
@@ -1015,6 +1026,16 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
 // host side
 // ---------------------------------------------------------------------------------------------
 
+// Programmatic dependent launch: the kernel may start (and run its set-up) while
+// the previous kernel on the stream finishes; it calls grid_dependency_wait()
+// before touching anything that kernel writes.  The quantizer does not signal
+// early, so a dependent GEMM starts only as the quantizer's last CTAs exit and
+// never holds SMs its predecessor still needs.
+void set_programmatic(cudaLaunchAttribute& a) {
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+}
+
 // Decode workspace after the 256-byte status block: one counter per 128-row
 // weight tile (rounded up to 256 bytes), then the FP32 partial tiles.
 size_t decode_counter_bytes(int64_t N) { return static_cast<size_t>(((N + 127) / 128 * 4 + 255) / 256 * 256); }
@@ -1121,13 +1142,14 @@ cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float
   cfg.blockDim = dim3(PairCfg::THREADS);
   cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  set_programmatic(attr[1]);
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tb, tsa, tsb, tc, a_gs, b_gs, static_cast<int>(M),
                             static_cast<int>(N), static_cast<int>(K), status);
 }
@@ -1161,10 +1183,17 @@ cudaError_t launch_decode(const uint8_t* a_codes, const uint8_t* a_sf, const flo
   // the counters were cleared together with the status word (gemm_zero_bytes)
   uint32_t* counters = reinterpret_cast<uint32_t*>(scratch);
   float* partial = reinterpret_cast<float*>(scratch + decode_counter_bytes(N));
-  gemm_decode_kernel<<<static_cast<unsigned>(G), DecodeCfg::THREADS, DecodeCfg::SMEM_BYTES, stream>>>(
-      tw, tx, b_sf, a_sf, a_gs, b_gs, c, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), ldc, max_seg,
-      partial, counters, status);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(G));
+  cfg.blockDim = dim3(DecodeCfg::THREADS);
+  cfg.dynamicSmemBytes = DecodeCfg::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  set_programmatic(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_decode_kernel, tw, tx, b_sf, a_sf, a_gs, b_gs, c, static_cast<int>(M),
+                            static_cast<int>(N), static_cast<int>(K), ldc, max_seg, partial, counters, status);
 }
 
 template <int BN>
@@ -1184,10 +1213,17 @@ cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + BN - 1) / BN);
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  gemm_kernel<BN><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, a_sf, b_sf, a_gs, b_gs, c,
-                                                                   static_cast<int>(M), static_cast<int>(N),
-                                                                   static_cast<int>(K), ldc, status);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  set_programmatic(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<BN>, ta, tb, a_sf, b_sf, a_gs, b_gs, c, static_cast<int>(M),
+                            static_cast<int>(N), static_cast<int>(K), ldc, status);
 }
 
 }  // namespace
@@ -1203,8 +1239,9 @@ size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
 }
 
 size_t gemm_zero_bytes(int64_t M, int64_t N, int64_t) {
-  // the status word, and for the decode kernel its tile counters right after the status block
-  return M <= DecodeCfg::BN ? 256 + decode_counter_bytes(N) : sizeof(uint32_t);
+  // the decode kernel's status word and tile counters; the tile kernels clear their
+  // status word themselves, so nothing separates them from the kernel before them
+  return M <= DecodeCfg::BN ? 256 + decode_counter_bytes(N) : 0;
 }
 
 cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,

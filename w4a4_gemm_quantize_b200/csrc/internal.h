@@ -31,9 +31,10 @@ cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
 // (split-K partial tiles of the small-M kernel); 0 when none.
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 
-// Bytes at the start of the workspace that must be zero when the GEMM launches (the
-// status word; for M <= 32 also the decode kernel's tile counters after the
-// 256-byte status block), cleared with one memset.
+// Bytes at the start of the workspace that must be zero when the GEMM launches:
+// for M <= 32 the decode kernel's status word and its tile counters after the
+// 256-byte status block (cleared with one memset); 0 for the tile kernels, which
+// clear their status word themselves.
 size_t gemm_zero_bytes(int64_t M, int64_t N, int64_t K);
 
 // Number of kernel launches the last call of each entry point enqueued (for

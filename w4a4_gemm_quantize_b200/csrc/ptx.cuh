@@ -90,6 +90,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Programmatic dependent launch: block until the grids this one was launched
+// behind have completed and their memory operations are visible (a no-op for a
+// launch without the programmatic-serialization attribute).  Everything a kernel
+// does before this call must not read what those grids write.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------------------------
 // TMA / bulk copies (global -> shared, completion counted on an mbarrier)
 // ---------------------------------------------------------------------------------------------

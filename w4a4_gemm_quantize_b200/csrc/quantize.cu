@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 1 ? 4 : 1) quantize_kernel(
     const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ gs_out, float* __restrict__ block_err) {
   __shared__ ScaleTables tab;
+  grid_dependency_wait();  // launched behind the amax pass (programmatic launch)
   const int64_t nblk = cols / 16;
   const int64_t atoms_per_group = (nblk + 3) / 4;
   const float sg = global_scale(gs_in, amax_bits);
@@ -348,6 +349,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const uint8_t* __r
                                                               const float* __restrict__ gs, int64_t rows,
                                                               int64_t cols, uint16_t* __restrict__ out,
                                                               int64_t ld_out) {
+  grid_dependency_wait();  // launched behind the kernel that wrote the codes (programmatic launch)
   const int64_t nblk = cols / 16;
   const int64_t total = rows * nblk;
   const int64_t atoms_per_group = (nblk + 3) / 4;
@@ -422,16 +424,24 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64
                             uint8_t* scales, float* gs_out, float* block_err, cudaStream_t stream) {
   const int64_t blocks16 = rows * (cols / 16);
   const int grid = grid_for(blocks16, kThreads);
-#define NVFP4_Q(MODE, SWZ)                                                                                 \
-  quantize_kernel<MODE, SWZ><<<grid, kThreads, 0, stream>>>(x, rows, cols, ld, gs_in, amax_bits, codes, \
-                                                            scales, gs_out, block_err)
-  if (mode == 1) {
-    if (swizzled) NVFP4_Q(1, true); else NVFP4_Q(1, false);
-  } else {
-    if (swizzled) NVFP4_Q(0, true); else NVFP4_Q(0, false);
-  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+#define NVFP4_Q(MODE, SWZ) \
+  cudaLaunchKernelEx(&cfg, quantize_kernel<MODE, SWZ>, x, rows, cols, ld, gs_in, amax_bits, codes, scales, gs_out, block_err)
+  cudaError_t e;
+  if (mode == 1)
+    e = swizzled ? NVFP4_Q(1, true) : NVFP4_Q(1, false);
+  else
+    e = swizzled ? NVFP4_Q(0, true) : NVFP4_Q(0, false);
 #undef NVFP4_Q
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_sf_pad_zero(uint8_t* scales, int64_t rows, int64_t nblk, cudaStream_t stream) {
@@ -449,11 +459,19 @@ cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStre
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, bool swizzled, const float* gs,
                               int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out, cudaStream_t stream) {
-  const int grid = grid_for(rows * (cols / 16), kThreads);
-  if (swizzled)
-    dequantize_kernel<true><<<grid, kThreads, 0, stream>>>(codes, scales, gs, rows, cols, out, ld_out);
-  else
-    dequantize_kernel<false><<<grid, kThreads, 0, stream>>>(codes, scales, gs, rows, cols, out, ld_out);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid_for(rows * (cols / 16), kThreads));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e =
+      swizzled ? cudaLaunchKernelEx(&cfg, dequantize_kernel<true>, codes, scales, gs, rows, cols, out, ld_out)
+               : cudaLaunchKernelEx(&cfg, dequantize_kernel<false>, codes, scales, gs, rows, cols, out, ld_out);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
