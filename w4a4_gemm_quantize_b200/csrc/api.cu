@@ -124,12 +124,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
     }
     return NVFP4_OK;
   }
-  if (swz) {
-    st = from_cuda(nvfp4::launch_sf_pad_zero(scales, rows, cols / 16, s));
-    if (st != NVFP4_OK) return st;
-    const int64_t rp = (rows + 127) / 128 * 128, cp = (cols / 16 + 3) / 4 * 4;
-    if (rp != rows || cp != cols / 16) ++nvfp4::g_last_launches;
-  }
+  // (the quantize kernel also zeroes the padding of a swizzled scale buffer)
   st = from_cuda(nvfp4::launch_quantize(static_cast<const uint16_t*>(x), rows, cols, ld_x, static_cast<int>(mode),
                                         swz, global_scale_in, amax_word, codes, scales, global_scale_out, block_err,
                                         s));

@@ -14,7 +14,6 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t l
 cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int mode,
                             bool swizzled, const float* gs_in, const uint32_t* amax_bits, uint8_t* codes,
                             uint8_t* scales, float* gs_out, float* block_err, cudaStream_t stream);
-cudaError_t launch_sf_pad_zero(uint8_t* scales, int64_t rows, int64_t nblk, cudaStream_t stream);
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, bool swizzled, const float* gs,
                               int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out, cudaStream_t stream);
 

@@ -190,6 +190,32 @@ __device__ __forceinline__ float global_scale(const float* gs_in, const uint32_t
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
 
+// Zero the padding of a swizzled scale buffer (rows [rows, Rp) and block columns
+// [nblk, Cp) of rows [0, rows)), grid-strided over all threads of the launch.
+__device__ __forceinline__ void zero_scale_padding(uint8_t* __restrict__ scales, int64_t rows, int64_t nblk) {
+  const int64_t rp = (rows + 127) / 128 * 128;
+  const int64_t cp = (nblk + 3) / 4 * 4;
+  const int64_t n_row_pad = (rp - rows) * cp;
+  const int64_t n_col_pad = rows * (cp - nblk);
+  if (n_row_pad + n_col_pad == 0) return;
+  const int64_t atoms_per_group = cp / 4;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_row_pad + n_col_pad;
+       i += stride) {
+    int64_t r, c;
+    if (i < n_row_pad) {
+      r = rows + i / cp;
+      c = i % cp;
+    } else {
+      const int64_t j = i - n_row_pad;
+      const int64_t wdt = cp - nblk;
+      r = j / wdt;
+      c = nblk + j % wdt;
+    }
+    scales[swizzled_offset(r, c, atoms_per_group)] = 0;
+  }
+}
+
 // The 127 finite non-negative E4M3 scale bytes of one tensor, decoded: eff =
 // RN32(dec(s) s_g) and RN32(1/eff) (0 for eff = 0).  Every CTA builds them once, so
 // each candidate scale costs two shared-memory reads instead of a conversion, a
@@ -203,7 +229,7 @@ struct ScaleTables {
 // fixed column chunk down the rows, so block coordinates and output offsets need
 // no division.
 template <int MODE, bool SWZ>
-__global__ void __launch_bounds__(kThreads, MODE == 1 ? 4 : 1) quantize_kernel(
+__global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, const float* __restrict__ gs_in,
     const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ gs_out, float* __restrict__ block_err) {
@@ -230,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 1 ? 4 : 1) quantize_kernel(
     r0 = w / chunks;
     c0 = w % chunks;
     c_step = chunks;
-    if (r0 >= r_step) return;  // the few warps past the last whole set of chunks
+    if (r0 >= r_step) r0 = rows;  // the few warps past the last whole set of chunks encode nothing
   } else {
     r0 = 0;
     r_step = 1;
@@ -316,31 +342,7 @@ __global__ void __launch_bounds__(kThreads, MODE == 1 ? 4 : 1) quantize_kernel(
       }
     }
   }
-}
-
-// Zero the padding of a swizzled scale buffer: rows [rows, Rp) and block columns
-// [nblk, Cp) of rows [0, rows).
-__global__ void sf_pad_zero_kernel(uint8_t* __restrict__ scales, int64_t rows, int64_t nblk) {
-  const int64_t rp = (rows + 127) / 128 * 128;
-  const int64_t cp = (nblk + 3) / 4 * 4;
-  const int64_t atoms_per_group = cp / 4;
-  const int64_t n_row_pad = (rp - rows) * cp;
-  const int64_t n_col_pad = rows * (cp - nblk);
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_row_pad + n_col_pad;
-       i += stride) {
-    int64_t r, c;
-    if (i < n_row_pad) {
-      r = rows + i / cp;
-      c = i % cp;
-    } else {
-      const int64_t j = i - n_row_pad;
-      const int64_t w = cp - nblk;
-      r = j / w;
-      c = nblk + j % w;
-    }
-    scales[swizzled_offset(r, c, atoms_per_group)] = 0;
-  }
+  if (SWZ) zero_scale_padding(scales, rows, nblk);
 }
 
 template <bool SWZ>
@@ -423,7 +425,11 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64
                             bool swizzled, const float* gs_in, const uint32_t* amax_bits, uint8_t* codes,
                             uint8_t* scales, float* gs_out, float* block_err, cudaStream_t stream) {
   const int64_t blocks16 = rows * (cols / 16);
-  const int grid = grid_for(blocks16, kThreads);
+  // enough threads for the larger of the blocks to encode and the padding to zero
+  // (a few activation rows pad their scales to 128 rows)
+  const int64_t nblk = cols / 16;
+  const int64_t pads = swizzled ? ((rows + 127) / 128 * 128) * ((nblk + 3) / 4 * 4) - blocks16 : 0;
+  const int grid = grid_for(blocks16 > pads ? blocks16 : pads, kThreads);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -442,14 +448,6 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64
     e = swizzled ? NVFP4_Q(0, true) : NVFP4_Q(0, false);
 #undef NVFP4_Q
   return e != cudaSuccess ? e : cudaGetLastError();
-}
-
-cudaError_t launch_sf_pad_zero(uint8_t* scales, int64_t rows, int64_t nblk, cudaStream_t stream) {
-  const int64_t rp = (rows + 127) / 128 * 128, cp = (nblk + 3) / 4 * 4;
-  const int64_t pads = (rp - rows) * cp + rows * (cp - nblk);
-  if (pads == 0) return cudaSuccess;
-  sf_pad_zero_kernel<<<grid_for(pads, kThreads), kThreads, 0, stream>>>(scales, rows, nblk);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t stream) {
