@@ -34,6 +34,7 @@ _LIB_PATH = os.path.join(_HERE, "libnvfp4_oracle.so")
 
 SCALE_ABSMAX = 0
 SCALE_MSE = 1
+SCALE_FOUR_OVER_SIX = 2
 
 _lib = None
 

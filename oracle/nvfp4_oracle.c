@@ -48,6 +48,11 @@
  *   R7 swizzled scale layout (the one the block-scaled tensor-core MMA reads):
  *      rows padded to 128, block columns padded to 4, zero fill; byte of
  *      (r, c) at ((r/128)*(Cp/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4.
+ *   R8 four-over-six: two candidates per block, the absmax scale (maximum
+ *      mapped to 6) first and s = E4M3(RN32(amax_b / RN32(4 s_g))) (maximum
+ *      mapped to 4) second, errors as in R5, the second kept only on a strict
+ *      improvement (ties keep the 6 mapping).  (parity unpinned: the order and
+ *      the tie rule are conventions; the pages name the choice, not its steps.)
  */
 #include <math.h>
 #include <stddef.h>
@@ -229,11 +234,17 @@ static float encode_block_with_eff(const float x[16], float eff, uint8_t codes[1
 
 #define ORA_SCALE_ABSMAX 0
 #define ORA_SCALE_MSE 1
+#define ORA_SCALE_FOUR_OVER_SIX 2
 
 /* Quantize one block of 16 (R2, R5).  Absmax: the single candidate f = 1, i.e.
  * s_b = E4M3(amax_b / (6 s_g)) -- s_absmax = max|W|/6 measured in units of s_g.
  * MSE: the candidates f = 0.3, 0.4, ..., 1.0 times the absmax scale, keeping
- * the least squared error (strict improvement while walking from f = 1 down). */
+ * the least squared error (strict improvement while walking from f = 1 down).
+ * Four-over-six ([G4] section 2, table of block-scale algorithms, row
+ * "Four-over-six": each block picks the larger of two possible maxima, 4 or 6,
+ * by least error): the absmax scale (block maximum mapped to 6), then
+ * s_b = E4M3(amax_b / (4 s_g)) (block maximum mapped to 4), kept only on a
+ * strictly smaller squared error (R8). */
 static uint8_t quantize_block(const float x[16], float sg, int mode, uint8_t codes[16],
                               float *err)
 {
@@ -257,6 +268,19 @@ static uint8_t quantize_block(const float x[16], float sg, int mode, uint8_t cod
         uint8_t c[16];
         float e = encode_block_with_eff(x, eff, c);
         if (i == 7 || e < best_e) {
+            best_e = e;
+            best_s = s;
+            memcpy(best_codes, c, 16);
+        }
+    }
+    if (mode == ORA_SCALE_FOUR_OVER_SIX) {
+        float d4 = 4.0f * sg;   /* RN32 (exact: a power of two) */
+        float v4 = amax_b / d4; /* RN32 */
+        uint8_t s = ora_e4m3_encode(v4);
+        float eff = (float)ora_e4m3_decode(s) * sg; /* RN32 */
+        uint8_t c[16];
+        float e = encode_block_with_eff(x, eff, c);
+        if (e < best_e) {
             best_e = e;
             best_s = s;
             memcpy(best_codes, c, 16);

@@ -296,6 +296,67 @@ def test_exhaustive_scale_search_bounds_mse():
             assert s_m[r, b] <= s_a[r, b] * (1 + 1e-5) + 1e-30
 
 
+# --- four-over-six (reading R8) ------------------------------------------------------------------
+
+
+def _blocks(rows):
+    """BF16 tensor from rows of 16 floats (each row one block)."""
+    return workloads.to_bf16(np.asarray(rows, np.float32))
+
+
+def test_four_over_six_picks_the_exact_4_mapping():
+    """A block whose maximum sits on 4 of the grid with every value on the E2M1 grid is exact
+    when its maximum maps to 4 (s_b = 1 with s_g = 1) and not when it maps to 6
+    (4/6 -> E4M3 0.6875, so 4 lands on 5.8 -> 6): four-over-six must take the 4 mapping,
+    absmax must not."""
+    vals = [4, 3, 2, 1.5, 1, 0.5, 0, -4, -3, -2, -1.5, -1, -0.5, 0, 4, 2]
+    x = _blocks([vals])
+    ca, sa, _, ea = oracle.quantize(x, oracle.SCALE_ABSMAX, sg=1.0)
+    cf, sf, _, ef = oracle.quantize(x, oracle.SCALE_FOUR_OVER_SIX, sg=1.0)
+    assert sa[0, 0] == 0x33 and ea[0, 0] > 0          # E4M3 0.6875 = 1.375 * 2^-1 (0 0110 011)
+    assert sf[0, 0] == 0x38 and ef[0, 0] == 0.0       # E4M3 1.0
+    grid = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    assert np.array_equal(grid[oracle.unpack_codes(cf)][0], np.asarray(vals, np.float64))
+
+
+def test_four_over_six_keeps_the_exact_6_mapping():
+    """A block exact with its maximum on 6 (s_b = 1): the 4 mapping (s_b = 1.5) puts 4 on
+    2.67 -> 3, so four-over-six keeps the absmax bits."""
+    x = _blocks([[6, 4, 3, 2, 1.5, 1, 0.5, 0, -6, -4, -3, -2, -1.5, -1, -0.5, 0]])
+    ca, sa, _, ea = oracle.quantize(x, oracle.SCALE_ABSMAX, sg=1.0)
+    cf, sf, _, ef = oracle.quantize(x, oracle.SCALE_FOUR_OVER_SIX, sg=1.0)
+    assert sa[0, 0] == 0x38 and ea[0, 0] == 0.0
+    assert np.array_equal(cf, ca) and np.array_equal(sf, sa) and ef[0, 0] == 0.0
+
+
+def test_four_over_six_ties_keep_the_6_mapping():
+    """All-zero and one-value blocks: both mappings give zero error, the 6 mapping stays."""
+    x = _blocks([[0.0] * 16, [0.0] * 15 + [3.0]])
+    ca, sa, sg, _ = oracle.quantize(x, oracle.SCALE_ABSMAX)
+    cf, sf, _, ef = oracle.quantize(x, oracle.SCALE_FOUR_OVER_SIX)
+    assert np.array_equal(sf, sa) and np.array_equal(cf, ca)
+
+
+def test_four_over_six_is_the_better_of_two_and_never_worse_than_absmax():
+    """Per block: the chosen scale is the absmax scale or E4M3(amax_b / (4 s_g)) (computed
+    here with torch's E4M3 conversion), its float64 error is the smaller of the two
+    mappings' (brute-force nearest-grid encode), and never above absmax."""
+    x = workloads.mse_weight(64, 256, seed=3)
+    ca, sa, sg, ea = oracle.quantize(x, oracle.SCALE_ABSMAX)
+    cf, sf, sg2, ef = oracle.quantize(x, oracle.SCALE_FOUR_OVER_SIX)
+    assert sg == sg2
+    assert np.all(ef <= ea)
+    xs = x.float().numpy().reshape(64, -1, 16)
+    amax = np.abs(xs).max(axis=2).astype(np.float32)
+    v4 = (amax / np.float32(np.float32(4) * np.float32(sg))).astype(np.float32)
+    s4 = torch.from_numpy(v4).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.all((sf == sa) | (sf == s4))
+    s_a, s_f = _sse64(x, ca, sa, sg), _sse64(x, cf, sf, sg)
+    assert np.all(s_f <= s_a * (1 + 1e-5) + 1e-30)
+    took4 = (sf == s4) & (sf != sa)
+    assert took4.sum() > 0 and (~took4).sum() > 0
+
+
 def test_toy_outlier_experiment_structure():
     """[DF] section 8: 4096 blocks of 16 from N(0, 0.02), one outlier per block scaled
     by 1, 3, 6, 12, 30.  The page prints no numbers; the search never loses to absmax
