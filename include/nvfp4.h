@@ -51,8 +51,12 @@ typedef enum {
  *  ABSMAX: s_b = E4M3(amax_b / (6 s_g)) -- the block's largest value lands on 6;
  *  MSE:    the candidates f * amax_b / (6 s_g), f = 0.3, 0.4, ..., 1.0, each
  *          rounded to E4M3; keep the one with the least squared reconstruction
- *          error sum_k (x_k - q_k s_b s_g)^2 (ties keep the larger scale). */
-typedef enum { NVFP4_SCALE_ABSMAX = 0, NVFP4_SCALE_MSE = 1 } nvfp4_scale_mode;
+ *          error sum_k (x_k - q_k s_b s_g)^2 (ties keep the larger scale);
+ *  FOUR_OVER_SIX: the same page's table of block-scale algorithms (section 2):
+ *          each block picks one of two maxima, 4 or 6, by least error -- the
+ *          absmax scale, then E4M3(amax_b / (4 s_g)) kept only on a strictly
+ *          smaller squared error (ties keep the absmax scale). */
+typedef enum { NVFP4_SCALE_ABSMAX = 0, NVFP4_SCALE_MSE = 1, NVFP4_SCALE_FOUR_OVER_SIX = 2 } nvfp4_scale_mode;
 
 /* Layout of the E4M3 block-scale buffer of a rows x cols tensor (nblk = cols/16).
  *  SWIZZLED: the 128 x 4 tiled layout that the tcgen05 block-scaled MMA reads
@@ -85,7 +89,7 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t cols);
 /* Quantize a BF16 matrix to NVFP4.
  *   x            device, BF16, rows x cols, row stride ld_x elements (ld_x >= cols, ld_x % 8 == 0).
  *   rows, cols   rows >= 0, cols % 16 == 0 (one scale per 16 values along a row).
- *   mode         NVFP4_SCALE_ABSMAX or NVFP4_SCALE_MSE.
+ *   mode         NVFP4_SCALE_ABSMAX, NVFP4_SCALE_MSE or NVFP4_SCALE_FOUR_OVER_SIX.
  *   layout       layout of `scales`.
  *   global_scale_in  device float or NULL.  NULL: s_g = amax(|x|) / 2688 (an
  *                all-zero tensor gets 1.0), computed on the device by a first

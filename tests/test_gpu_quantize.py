@@ -16,7 +16,8 @@ import w4a4_gemm_quantize_b200 as nv
 
 pytestmark = pytest.mark.gpu
 
-MODES = {"absmax": oracle.SCALE_ABSMAX, "mse": oracle.SCALE_MSE}
+MODES = {"absmax": oracle.SCALE_ABSMAX, "mse": oracle.SCALE_MSE, "four_over_six": oracle.SCALE_FOUR_OVER_SIX}
+ALL_MODES = list(MODES)
 
 
 def _f32_bits(v):
@@ -62,7 +63,7 @@ def _first_diff(a, b):
 
 # --- the pages' workloads -----------------------------------------------------------------------
 
-@pytest.mark.parametrize("mode", ["absmax", "mse"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 @pytest.mark.parametrize("layout", ["swizzled", "linear"])
 def test_pr1_reference_config(cuda_device, mode, layout):
     d = workloads.pr1(seed=0)
@@ -70,7 +71,7 @@ def test_pr1_reference_config(cuda_device, mode, layout):
     run_and_compare(d["x"], mode, layout)
 
 
-@pytest.mark.parametrize("mode", ["absmax", "mse"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_mse_workload_small_full_compare(cuda_device, mode):
     """0.02 * Student-t(3), 8 x 128-row tiles with a ragged tail of rows."""
     run_and_compare(workloads.mse_weight(1000, 1024, seed=1), mode)
@@ -83,6 +84,18 @@ def test_mse_workload_full_size_sampled(cuda_device, mode):
     rows = np.unique(np.concatenate([np.arange(0, 4), np.arange(4090, 4096),
                                      np.random.default_rng(0).choice(4096, 48, replace=False)]))
     run_and_compare(x, mode, rows_sample=rows)
+
+
+def test_four_over_six_blocks_exact_on_one_mapping(cuda_device):
+    """Blocks on the E2M1 grid with their maximum on 4 (exact only when the maximum maps to 4)
+    and on 6 (exact only when it maps to 6), a zero block and a one-value tie, with s_g = 1:
+    the GPU takes the 4 mapping exactly where the oracle does."""
+    b4 = [4, 3, 2, 1.5, 1, 0.5, 0, -4, -3, -2, -1.5, -1, -0.5, 0, 4, 2]
+    b6 = [6, 4, 3, 2, 1.5, 1, 0.5, 0, -6, -4, -3, -2, -1.5, -1, -0.5, 0]
+    a = np.array([b4 + b6, b6 + b4, [0.0] * 16 + [0.0] * 15 + [3.0], [x * 0.25 for x in b4] + b4], np.float32)
+    q = run_and_compare(workloads.to_bf16(a), "four_over_six", sg=1.0)
+    lin = oracle.unswizzle_scales(q.scales.cpu().numpy(), 4, 2)
+    assert lin[0, 0] == 0x38 and lin[1, 1] == 0x38  # E4M3 1.0: the block maximum 4 maps to 4
 
 
 def test_decode_activations_outlier_channels(cuda_device):
@@ -104,7 +117,7 @@ def test_prefill_activation_sampled(cuda_device):
 
 # --- edge cases ---------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("mode", ["absmax", "mse"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_edge_values(cuda_device, mode):
     r = np.random.default_rng(5)
     a = (r.standard_t(3, size=(130, 48)) * 0.02).astype(np.float32)
@@ -118,7 +131,7 @@ def test_edge_values(cuda_device, mode):
     run_and_compare(workloads.to_bf16(a), mode)
 
 
-@pytest.mark.parametrize("mode", ["absmax", "mse"])
+@pytest.mark.parametrize("mode", ALL_MODES)
 def test_huge_and_tiny_magnitudes(cuda_device, mode):
     """A BF16 value near the format maximum next to ordinary and subnormal values:
     most block scales underflow to E4M3 zero; tiny tensors push s_g to subnormal."""
@@ -139,14 +152,14 @@ def test_rounding_midpoints_with_given_global_scale(cuda_device):
     mids = np.array([6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, 5.5, 6.5, 0.2, 0.3, 2.75, 4.5, 1.0, 0.5],
                     np.float32) * np.float32(0.125)
     a = np.stack([mids, -mids, mids[::-1].copy(), np.roll(mids, 3)])
-    for mode in ("absmax", "mse"):
+    for mode in ALL_MODES:
         run_and_compare(workloads.to_bf16(a), mode, sg=0.125)
 
 
 @pytest.mark.parametrize("shape", [(1, 16), (3, 32), (127, 16), (128, 64), (129, 80), (257, 272)])
 def test_ragged_shapes(cuda_device, shape):
     a = np.random.default_rng(sum(shape)).standard_normal(shape).astype(np.float32)
-    for mode in ("absmax", "mse"):
+    for mode in ALL_MODES:
         for layout in ("swizzled", "linear"):
             run_and_compare(workloads.to_bf16(a), mode, layout)
 

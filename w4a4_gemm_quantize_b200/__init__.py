@@ -27,10 +27,12 @@ LIB_PATH = os.path.join(_HERE, "libnvfp4_b200.so")
 
 SCALE_ABSMAX = 0
 SCALE_MSE = 1
+SCALE_FOUR_OVER_SIX = 2
 SF_SWIZZLED = 0
 SF_LINEAR = 1
 
-_MODES = {"absmax": SCALE_ABSMAX, "mse": SCALE_MSE, SCALE_ABSMAX: SCALE_ABSMAX, SCALE_MSE: SCALE_MSE}
+_MODES = {"absmax": SCALE_ABSMAX, "mse": SCALE_MSE, "four_over_six": SCALE_FOUR_OVER_SIX,
+          SCALE_ABSMAX: SCALE_ABSMAX, SCALE_MSE: SCALE_MSE, SCALE_FOUR_OVER_SIX: SCALE_FOUR_OVER_SIX}
 _LAYOUTS = {"swizzled": SF_SWIZZLED, "linear": SF_LINEAR, SF_SWIZZLED: SF_SWIZZLED, SF_LINEAR: SF_LINEAR}
 
 STATUS = {0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_SHAPE", 3: "NVFP4_ERR_ALIGNMENT",

@@ -78,7 +78,8 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
                             void* stream) {
   nvfp4::g_last_launches = 0;
   if (rows < 0 || cols < 0 || ld_x < cols) return NVFP4_ERR_INVALID_ARG;
-  if (mode != NVFP4_SCALE_ABSMAX && mode != NVFP4_SCALE_MSE) return NVFP4_ERR_INVALID_ARG;
+  if (mode != NVFP4_SCALE_ABSMAX && mode != NVFP4_SCALE_MSE && mode != NVFP4_SCALE_FOUR_OVER_SIX)
+    return NVFP4_ERR_INVALID_ARG;
   if (layout != NVFP4_SF_SWIZZLED && layout != NVFP4_SF_LINEAR) return NVFP4_ERR_INVALID_ARG;
   if (cols % 16 != 0) return NVFP4_ERR_SHAPE;
   if (rows == 0 || cols == 0) {

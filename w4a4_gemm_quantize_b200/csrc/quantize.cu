@@ -18,6 +18,9 @@
 //   y_k = |x_k| r, mag_k = E2M1_sat(y_k) (RNE), code_k = sign(x_k) | mag_k;
 //   block error e = fma(d_k, d_k, e) over k with d_k = fma(-|q_k|, eff, |x_k|);
 //   candidates walked from f = 1 down, kept on a strict improvement.
+//  * four-over-six (same page, section 2, table of block-scale algorithms: each
+//    block picks one of two maxima, 4 or 6, by least error): the absmax scale,
+//    then s_b = E4M3(amax_b / (4 s_g)) kept only on a strictly smaller error.
 //
 // Kernels are HBM-bound streaming kernels (absmax) or ALU-bound (MSE): one
 // thread per 16-value block, 2 x 128-bit loads per thread, packed 8-byte code
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
         uint32_t best_c0, best_c1;
         encode_codes(x2, best_eff, tab.rcp[best_s], best_c0, best_c1);
         float best_e = 0.0f;
-        if (MODE == 1 || block_err) best_e = block_sse(x2, best_c0, best_c1, best_eff);
+        if (MODE != 0 || block_err) best_e = block_sse(x2, best_c0, best_c1, best_eff);
 
         if (MODE == 1) {
           const float factors[7] = {0.9f, 0.8f, 0.7f, 0.6f, 0.5f, 0.4f, 0.3f};
@@ -318,6 +321,22 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
             uint32_t c0w, c1w;
             encode_codes(x2, eff, rcp, c0w, c1w);
             const float e = block_sse(x2, c0w, c1w, eff);
+            if (e < best_e) {
+              best_e = e;
+              best_s = s;
+              best_c0 = c0w;
+              best_c1 = c1w;
+            }
+          }
+        }
+        if (MODE == 2) {
+          // four-over-six: the block maximum mapped to 4 instead of 6, kept only on a
+          // strictly smaller error (4 s_g is exact: a power-of-two multiple)
+          const uint32_t s = cvt_e4m3_satfinite(__fdiv_rn(amax_b, __fmul_rn(4.0f, sg)));
+          if (s != best_s) {
+            uint32_t c0w, c1w;
+            encode_codes(x2, tab.eff[s], tab.rcp[s], c0w, c1w);
+            const float e = block_sse(x2, c0w, c1w, tab.eff[s]);
             if (e < best_e) {
               best_e = e;
               best_s = s;
@@ -442,7 +461,9 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64
 #define NVFP4_Q(MODE, SWZ) \
   cudaLaunchKernelEx(&cfg, quantize_kernel<MODE, SWZ>, x, rows, cols, ld, gs_in, amax_bits, codes, scales, gs_out, block_err)
   cudaError_t e;
-  if (mode == 1)
+  if (mode == 2)
+    e = swizzled ? NVFP4_Q(2, true) : NVFP4_Q(2, false);
+  else if (mode == 1)
     e = swizzled ? NVFP4_Q(1, true) : NVFP4_Q(1, false);
   else
     e = swizzled ? NVFP4_Q(0, true) : NVFP4_Q(0, false);
