@@ -66,6 +66,8 @@ def test_quantize_validation_before_any_cuda_call(lib):
     assert _q(lib, rows=-1) == 1                    # negative size
     assert _q(lib, ld=16) == 1                      # ld < cols
     assert _q(lib, mode=5) == 1                     # unknown mode
+    assert _q(lib, mode=3) == 1
+    assert _q(lib, mode=2) in (4, 5)                # four-over-six is a valid mode
     assert _q(lib, layout=7) == 1                   # unknown layout
     assert _q(lib, x=0) == 1                        # NULL input
     assert _q(lib, ws=0) == 7                       # no workspace, no global scale
@@ -98,6 +100,27 @@ def test_gemm_validation_before_any_cuda_call(lib):
     assert need > 256
     assert g(M=8, N=14336, ldc=14336, K=4096) == 7
     assert g(M=8, N=14336, ldc=14336, K=4096, ws_bytes=need) in (4, 5)
+    assert g(M=8, N=14336, ldc=14336, K=4096, ws_bytes=need - 1) == 7
+
+
+def test_decode_workspace_holds_every_partial_tile():
+    """M <= 32: the weight stream (128-row tiles x 256-wide K-tiles) is split evenly over
+    up to 296 CTAs; a tile spans at most (KT - 1) // per + 2 CTA ranges (per = units per
+    CTA, rounded down), each with a 128 x 32 FP32 partial slot, after the 256-byte status
+    block and one counter word per tile (rounded up to 256 bytes)."""
+    lib = nv.load_library()
+    for (M, N, K) in [(8, 14336, 4096), (1, 21504, 5376), (32, 5376, 21504), (2, 384, 8192), (24, 1000, 2080),
+                      (1, 128, 32)]:
+        T, KT = -(-N // 128), -(-K // 256)
+        U = T * KT
+        G = min(296, U)
+        per = max(1, U // G)
+        segs = min(KT, (KT - 1) // per + 2)
+        counters = -(-(T * 4) // 256) * 256
+        assert lib.nvfp4_gemm_workspace_bytes(M, N, K) == 256 + counters + T * segs * 128 * 32 * 4, (M, N, K)
+    # larger M needs only the status block
+    assert lib.nvfp4_gemm_workspace_bytes(33, 14336, 4096) == 256
+    assert lib.nvfp4_gemm_workspace_bytes(8192, 21504, 5376) == 256
 
 
 def test_dequantize_validation(lib):
