@@ -279,7 +279,7 @@ def work_units(cfg):
 def gemm_kernel_name(M: int, N: int) -> str:
     """The kernel the library picks for an M x N output (its launch dispatch)."""
     if M <= 32:
-        return "gemm_decode_kernel (tcgen05 mxf4nvf4, split-K)"
+        return "gemm_decode_kernel (tcgen05 mxf4nvf4, stream-K)"
     if M > 128 and N > 128:
         return "gemm_pair_kernel (tcgen05 cta_group::2 mxf4nvf4)"
     return "gemm_kernel (tcgen05 mxf4nvf4)"

@@ -95,7 +95,7 @@ def test_gemm_validation_before_any_cuda_call(lib):
     assert g(ldc=20) == 3
     assert g(gs=2) == 3
     assert g() in (4, 5)
-    # small M uses split-K scratch after the status word: a 256-byte workspace is too small
+    # small M uses stream-K scratch after the status word: a 256-byte workspace is too small
     need = lib.nvfp4_gemm_workspace_bytes(8, 14336, 4096)
     assert need > 256
     assert g(M=8, N=14336, ldc=14336, K=4096) == 7

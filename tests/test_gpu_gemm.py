@@ -85,9 +85,10 @@ def test_more_tiles_than_sms_full_compare(cuda_device, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(24, 1000, 2080), (2, 384, 8192), (32, 14336, 512)])
-def test_small_m_split_k_full_compare(cuda_device, M, N, K):
-    """The small-M kernel (weights on the 128-row MMA side) with K split over several
-    CTAs: ragged N, a partial last K-tile, and the slice reduction."""
+def test_small_m_stream_k_full_compare(cuda_device, M, N, K):
+    """The small-M kernel (weights on the 128-row MMA side, the weight stream split evenly
+    over the SMs): ragged N, a partial last K-tile, tiles cut into up to 32 segments
+    (N=384, K=8192: one K-tile per CTA) and the ordered partial reduction."""
     xa = workloads.activation(M, K, seed=M + 7, n_outlier_channels=2)
     xb = workloads.gaussian_weight(N, K, 0.02, seed=N + 7)
     run_full(oracle_operand(xa), oracle_operand(xb, oracle.SCALE_MSE), M, N, K)
