@@ -99,6 +99,8 @@ def _load():
     lib.ora_e4m3_encode_array.restype = None
     lib.ora_f32_to_bf16_array.argtypes = [P, I64, P]
     lib.ora_f32_to_bf16_array.restype = None
+    lib.ora_lora_f64.argtypes = [P, I64, I64, P, I64, P, I64, P, P, P]
+    lib.ora_lora_f64.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -273,6 +275,25 @@ def gemm_f64_at(a_codes, a_scales, a_sg, b_codes, b_scales, b_sg, m_idx, n_idx):
     if rc != 0:
         raise MemoryError("oracle GEMM work buffer")
     return out, absum
+
+
+def lora_f64(x, a, b):
+    """Low-rank term of y = W_4bit x + B (A x) (reading R9): x (M, K), a (R, K), b (N, R) BF16.
+
+    Returns (u [M, N] float64, S_u = sum |t b| [M, N], t [M, R] BF16 bits) with
+    t = BF16_RNE(RN32(x a^T)) and u = t b^T in binary64."""
+    x, a, b = _bits(x), _bits(a), _bits(b)
+    M, K = x.shape
+    R = a.shape[0]
+    N = b.shape[0]
+    assert a.shape[1] == K and b.shape[1] == R
+    out = np.empty((M, N), np.float64)
+    absum = np.empty((M, N), np.float64)
+    t = np.empty((M, R), np.uint16)
+    rc = _load().ora_lora_f64(_ptr(x), M, K, _ptr(a), R, _ptr(b), N, _ptr(out), _ptr(absum), _ptr(t))
+    if rc != 0:
+        raise MemoryError("oracle LoRA work buffer")
+    return out, absum, t
 
 
 def unpack_codes(codes: np.ndarray) -> np.ndarray:

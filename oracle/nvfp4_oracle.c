@@ -48,6 +48,13 @@
  *   R7 swizzled scale layout (the one the block-scaled tensor-core MMA reads):
  *      rows padded to 128, block columns padded to 4, zero fill; byte of
  *      (r, c) at ((r/128)*(Cp/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4.
+ *   R9 LoRA branch ([DF] section 3, "¿Cómo fine-tuneás algo que ya está en 4
+ *      bits?": y = W_4bit x + B (A x), the low-rank term in 16 bits, added to the
+ *      quantized matmul before the result is returned): x is the activation
+ *      before quantization (BF16), A (r x K) and B (N x r) are BF16; the
+ *      intermediate t = A x is rounded to BF16 (the 16-bit term), the sums are
+ *      binary64 here; the W4A4 accumulator plus the low-rank term is rounded to
+ *      BF16 once.  (parity unpinned: where the 16-bit rounding happens is a reading.)
  *   R8 four-over-six: two candidates per block, the absmax scale (maximum
  *      mapped to 6) first and s = E4M3(RN32(amax_b / RN32(4 s_g))) (maximum
  *      mapped to 4) second, errors as in R5, the second kept only on a strict
@@ -474,4 +481,48 @@ void ora_f32_to_bf16_array(const float *f, int64_t n, uint16_t *out)
 {
     for (int64_t i = 0; i < n; i++)
         out[i] = ora_f32_to_bf16(f[i]);
+}
+
+/* ------------------------------------------------------------------------- */
+/* LoRA branch (R9): the low-rank term of y = W_4bit x + B (A x).             */
+/* ------------------------------------------------------------------------- */
+
+/* x: M x K BF16 bits (row stride K); a: R x K; b: N x R (both BF16 bits).
+ * t_out (M x R BF16 bits, optional): t = BF16_RNE(RN32(sum_k x[m][k] a[j][k])).
+ * out (M x N): out[m][n] = sum_j t[m][j] b[n][j] in binary64; absum: the sum of
+ * the terms' magnitudes.  Returns 0, or -1 on a bad size or allocation. */
+int ora_lora_f64(const uint16_t *x, int64_t M, int64_t K, const uint16_t *a, int64_t R, const uint16_t *b,
+                 int64_t N, double *out, double *absum, uint16_t *t_out)
+{
+    if (M < 0 || K < 0 || R < 0 || N < 0)
+        return -1;
+    double *t = (double *)malloc(sizeof(double) * (size_t)(M * R + 1));
+    if (!t)
+        return -1;
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t j = 0; j < R; j++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += (double)ora_bf16_to_f32(x[m * K + k]) * (double)ora_bf16_to_f32(a[j * K + k]);
+            /* the 16-bit intermediate: BF16_RNE(RN32(acc)), the rounding a binary32
+             * accumulator followed by a BF16 store performs */
+            uint16_t tb = ora_f32_to_bf16((float)acc);
+            if (t_out)
+                t_out[m * R + j] = tb;
+            t[m * R + j] = (double)ora_bf16_to_f32(tb);
+        }
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t j = 0; j < R; j++) {
+                double p = t[m * R + j] * (double)ora_bf16_to_f32(b[n * R + j]);
+                acc += p;
+                mag += fabs(p);
+            }
+            out[m * N + n] = acc;
+            if (absum)
+                absum[m * N + n] = mag;
+        }
+    free(t);
+    return 0;
 }

@@ -357,6 +357,77 @@ def test_four_over_six_is_the_better_of_two_and_never_worse_than_absmax():
     assert took4.sum() > 0 and (~took4).sum() > 0
 
 
+# --- LoRA branch (reading R9) ----------------------------------------------------------------------
+
+
+def _bf16_rand(shape, scale, seed):
+    return workloads.to_bf16(np.random.default_rng(seed).standard_normal(shape).astype(np.float32) * scale)
+
+
+def test_lora_exact_integer_case():
+    """Small integers (exact in BF16, products and sums exact, t below 256 so exact in BF16):
+    the low-rank term equals the integer matmul B (A x) exactly."""
+    r = np.random.default_rng(9)
+    x = r.integers(-3, 4, size=(5, 24))
+    a = r.integers(-2, 3, size=(4, 24))
+    b = r.integers(-3, 4, size=(7, 4))
+    t_int = x @ a.T
+    assert np.abs(t_int).max() < 256
+    u, s_u, t = oracle.lora_f64(workloads.to_bf16(x.astype(np.float32)), workloads.to_bf16(a.astype(np.float32)),
+                                workloads.to_bf16(b.astype(np.float32)))
+    assert np.array_equal(u, (t_int @ b.T).astype(np.float64))
+    assert np.array_equal(s_u, (np.abs(t_int)[:, None, :] * np.abs(b)[None, :, :]).sum(axis=2).astype(np.float64))
+
+
+def test_lora_intermediate_is_the_bf16_rounded_product():
+    """The 16-bit intermediate t is torch's BF16 rounding of the binary32 rounding of A x
+    (computed here in float64 by numpy), and u = t B^T."""
+    x, a, b = _bf16_rand((6, 96), 1.0, 1), _bf16_rand((16, 96), 0.05, 2), _bf16_rand((40, 16), 0.05, 3)
+    u, _, t = oracle.lora_f64(x, a, b)
+    xf, af, bf = (v.float().numpy().astype(np.float64) for v in (x, a, b))
+    t_ref = torch.from_numpy((xf @ af.T).astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(t, t_ref.view(torch.int16).numpy().view(np.uint16))
+    tf = t_ref.float().numpy().astype(np.float64)
+    assert np.allclose(u, tf @ bf.T, rtol=1e-12, atol=1e-15)
+    assert not np.array_equal(tf, xf @ af.T)  # the rounding is visible at this size
+
+
+def test_lora_zero_rank_or_zero_b_adds_nothing():
+    x, a = _bf16_rand((3, 32), 1.0, 4), _bf16_rand((8, 32), 0.1, 5)
+    u, s_u, _ = oracle.lora_f64(x, a, workloads.to_bf16(np.zeros((10, 8), np.float32)))
+    assert not u.any() and not s_u.any()
+    u0, s0, t0 = oracle.lora_f64(x, a[:0], workloads.to_bf16(np.zeros((10, 0), np.float32)))
+    assert u0.shape == (3, 10) and not u0.any() and t0.shape == (3, 0)
+
+
+def test_merging_a_lora_into_nvfp4_erases_most_of_it():
+    """[DF] section 3: in a block whose scale is 0.01 the weights can only be 0, +-0.005,
+    +-0.01, +-0.015, +-0.02, +-0.03, +-0.04, +-0.06; a LoRA correction of about 0.001 is a
+    tenth of a step, so merging it and quantizing again rounds the correction away.  With
+    the block scale exactly 0.01, weights on those levels plus +-0.001 re-quantize to the
+    same values everywhere (only the sign of some zeros changes), while the fused low-rank
+    branch keeps the term."""
+    levels = np.array([0, 0.005, 0.01, 0.015, 0.02, 0.03, 0.04, 0.06], np.float32)
+    r = np.random.default_rng(12)
+    w = (r.choice(levels, size=(64, 64)) * r.choice([-1, 1], size=(64, 64))).astype(np.float32)
+    w[:, ::16] = 0.06                                  # every block's maximum maps to 6: s_b s_g = 0.01
+    sg = np.float32(0.01) / np.float32(1.0)            # block scale 1.0 (E4M3 exact), eff = RN32(0.01)
+    delta = (r.choice([-1, 1], size=w.shape) * 0.001).astype(np.float32)
+    c0, s0, _, _ = oracle.quantize(workloads.to_bf16(w), oracle.SCALE_ABSMAX, sg=sg)
+    c1, s1, _, _ = oracle.quantize(workloads.to_bf16(w + delta), oracle.SCALE_ABSMAX, sg=sg)
+    assert np.all(s0 == 0x38) and np.array_equal(s0, s1)
+    grid = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    q0, q1 = grid[oracle.unpack_codes(c0)], grid[oracle.unpack_codes(c1)]
+    assert np.array_equal(q0, q1)                      # every correction rounded away
+    # the fused low-rank branch keeps it: a rank-1 branch (A = one row of the correction,
+    # B = ones) gives a non-zero B (A x)
+    x = workloads.to_bf16(np.ones((1, 64), np.float32))
+    a = workloads.to_bf16(delta[:1])                   # r = 1, K = 64
+    b = workloads.to_bf16(np.ones((64, 1), np.float32))
+    u, _, _ = oracle.lora_f64(x, a, b)
+    assert np.all(u != 0)
+
+
 def test_toy_outlier_experiment_structure():
     """[DF] section 8: 4096 blocks of 16 from N(0, 0.02), one outlier per block scaled
     by 1, 3, 6, 12, 30.  The page prints no numbers; the search never loses to absmax
