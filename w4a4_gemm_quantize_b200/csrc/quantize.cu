@@ -10,7 +10,10 @@
 //    s = max|x| / 6, or the MSE scale that minimises sum_k (x_k - s s_g Q(x_k/(s s_g)))^2
 //    over candidates below the absmax scale (the search of section 8 "Para
 //    practicar" of "NVFP4 en difusión: la misma cuantización, un motor
-//    completamente distinto", with 8 factors 0.3, 0.4, ..., 1.0).
+//    completamente distinto", with 8 factors 0.3, 0.4, ..., 1.0);
+//  * the section's table of block-scale algorithms, row "Four-over-six": each
+//    block picks one of two maxima, 4 or 6, by least error -- the absmax scale,
+//    then s_b = E4M3(amax_b / (4 s_g)) kept only on a strictly smaller error.
 //
 // Arithmetic, in this order and all binary32 round-to-nearest-even:
 //   s_g = amax_t / 2688 (1 for an all-zero tensor); d6 = 6 s_g; v_b = amax_b / d6;
@@ -18,13 +21,14 @@
 //   y_k = |x_k| r, mag_k = E2M1_sat(y_k) (RNE), code_k = sign(x_k) | mag_k;
 //   block error e = fma(d_k, d_k, e) over k with d_k = fma(-|q_k|, eff, |x_k|);
 //   candidates walked from f = 1 down, kept on a strict improvement.
-//  * four-over-six (same page, section 2, table of block-scale algorithms: each
-//    block picks one of two maxima, 4 or 6, by least error): the absmax scale,
-//    then s_b = E4M3(amax_b / (4 s_g)) kept only on a strictly smaller error.
 //
-// Kernels are HBM-bound streaming kernels (absmax) or ALU-bound (MSE): one
-// thread per 16-value block, 2 x 128-bit loads per thread, packed 8-byte code
-// stores; hardware cvt for E4M3 and E2M1 rounding.
+// Kernels: the absmax pass is HBM-bound, the MSE search issue-bound.  One thread
+// per 16-value block (2 x 128-bit loads, packed 8-byte code stores), one warp per
+// 32 consecutive blocks of a row, per-CTA tables of the decoded scales and their
+// reciprocals, hardware cvt for E4M3 and E2M1 rounding, swizzled scale bytes
+// stored four at a time; the encode kernel also zeroes the swizzled padding.
+// Every kernel is launched with programmatic dependent launch and waits for its
+// predecessor before reading its inputs.
 #include <cuda_runtime.h>
 
 #include "internal.h"
