@@ -141,3 +141,33 @@ def test_selftest_validation(lib):
     assert lib.nvfp4_selftest_wait_timeout(P(16), 0, None) == 1
     assert lib.nvfp4_selftest_wait_timeout(P(16), 3000000, None) == 1
     assert lib.nvfp4_selftest_wait_timeout(P(8), 1000, None) == 3
+
+
+def test_binding_constants_match_the_header():
+    """The Python binding's enum values and status names are the ones include/nvfp4.h
+    declares (parsed from the header text)."""
+    hdr = open(HEADER).read()
+    enum = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(NVFP4_[A-Z0-9_]+)\s*=\s*(\d+)", hdr)}
+    assert enum["NVFP4_SCALE_ABSMAX"] == nv.SCALE_ABSMAX
+    assert enum["NVFP4_SCALE_MSE"] == nv.SCALE_MSE
+    assert enum["NVFP4_SCALE_FOUR_OVER_SIX"] == nv.SCALE_FOUR_OVER_SIX
+    assert enum["NVFP4_SF_SWIZZLED"] == nv.SF_SWIZZLED and enum["NVFP4_SF_LINEAR"] == nv.SF_LINEAR
+    status = {v: k for k, v in enum.items() if k == "NVFP4_OK" or k.startswith("NVFP4_ERR_")}
+    assert status == nv.STATUS
+
+
+def test_bench_profile_record_matches_only_its_sources(tmp_path, monkeypatch):
+    """bench.py reports the ncu DRAM traffic of a profile summary only while the summary's
+    source hash equals the hash of the kernel's current sources."""
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    real_csrc = os.path.join(os.path.dirname(os.path.abspath(bench.__file__)), "w4a4_gemm_quantize_b200", "csrc")
+    os.makedirs(tmp_path / "w4a4_gemm_quantize_b200")
+    os.symlink(real_csrc, tmp_path / "w4a4_gemm_quantize_b200" / "csrc")
+    os.makedirs(tmp_path / "profiles")
+    h = bench.source_hash("gemm")
+    (tmp_path / "profiles" / "gemm_w.md").write_text(f"- source_hash: `{h}`\n- traffic_bytes_per_launch: 1234\n")
+    assert bench.profiled_traffic("gemm", "w") == 1234.0
+    (tmp_path / "profiles" / "gemm_w.md").write_text("- source_hash: `0000000000000000`\n- traffic_bytes_per_launch: 1234\n")
+    assert bench.profiled_traffic("gemm", "w") is None
+    assert bench.profiled_traffic("gemm", "missing") is None
