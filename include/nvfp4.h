@@ -147,8 +147,46 @@ nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const f
                         const float *b_global_scale, int64_t N, int64_t K, void *c, int64_t ldc,
                         void *workspace, size_t workspace_bytes, void *stream);
 
+/* Workspace nvfp4_linear needs (device memory, any content on entry): 512 bytes
+ * (status word, the activation's amax and global scale), plus for M <= 32 the
+ * small-M kernel's tile counters and partial tiles, for M > 32 the activation's
+ * codes and swizzled scales. */
+size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* The W4A4 linear layer: the BF16 activation X is quantized on this call (absmax
+ * block scales) and multiplied by the pre-quantized weight W, C = Q(X) W^T in BF16
+ * -- the page "NVFP4 en difusión: la misma cuantización, un motor completamente
+ * distinto", section 2 "NVFP4 sin vLLM: torch._scaled_mm a mano" (the activation
+ * is quantized on every forward, 16-block by 16-block, while the weights come
+ * quantized from the checkpoint; out = (A s_a)(B s_b)^T in BF16), with the
+ * quantization done in the same kernel as the matmul where the activation is small,
+ * as section 3 describes for nunchaku's fused kernel.
+ *   x            device, BF16, M x K, row stride ld_x elements (ld_x >= K, ld_x % 8 == 0).
+ *   x_global_scale  device float or NULL: the activation's per-tensor FP32 scale.
+ *                Given (a calibrated activation scale: "Tu pipeline NVFP4 ...",
+ *                section 2, the third of the "three questions" every quantization
+ *                scheme answers -- activation scales come from calibration on real
+ *                activations), nothing reads the whole of x first.  NULL:
+ *                s_g = amax(|x|) / 2688 computed on the device by a first pass, as
+ *                nvfp4_quantize does.
+ *   w_codes, w_scales, w_global_scale  the weight N x K as nvfp4_quantize writes it
+ *                (scales SWIZZLED).
+ *   c            device BF16, M x N, row stride ldc (ldc >= N, ldc % 8 == 0).
+ *   M, N >= 1; K >= 32, K % 32 == 0.
+ * The result equals nvfp4_quantize(x, ABSMAX, SWIZZLED, x_global_scale) followed by
+ * nvfp4_gemm bit for bit.  For M <= 32 one kernel quantizes the activation K-tiles
+ * it consumes and multiplies (plus the amax pass when x_global_scale is NULL); for
+ * M > 32 the quantizer writes the activation's codes into the workspace and the
+ * GEMM reads them (kernels chained with programmatic dependent launch).
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, WORKSPACE, UNSUPPORTED_DEVICE, CUDA; a
+ * device-side timeout is read with nvfp4_read_device_error(workspace, ...). */
+nvfp4_status nvfp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, const float *x_global_scale,
+                          const uint8_t *w_codes, const uint8_t *w_scales, const float *w_global_scale,
+                          int64_t N, void *c, int64_t ldc, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
 /* Synchronize `stream` and read the device status word at the start of a GEMM
- * workspace.  Returns NVFP4_OK when no bounded wait gave up, NVFP4_ERR_TIMEOUT
+ * (or nvfp4_linear) workspace.  Returns NVFP4_OK when no bounded wait gave up, NVFP4_ERR_TIMEOUT
  * otherwise (and stores the raw word, which names the wait, in *word if non-NULL),
  * NVFP4_ERR_CUDA if the copy fails.  Clears nothing: a workspace is reset by the
  * next nvfp4_gemm that uses it. */
@@ -173,7 +211,9 @@ nvfp4_status nvfp4_selftest_wait_timeout(void *workspace, uint32_t timeout_us, v
  *  - It allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
  *  - The first call on a device, with that device current, looks up the scratch
  *    block's device address (cudaGetSymbolAddress); make that first call before
- *    any stream capture.
+ *    any stream capture.  The address is cached per device and CUDA context: after
+ *    cudaDeviceReset (which frees the block with the context) the next call looks
+ *    it up again in the new context, so make that call outside a capture too.
  *  - Every call shares the one scratch block per device and clears what it needs
  *    zeroed before use; calls whose work overlaps on the GPU (other streams, or
  *    other host threads) race on it -- serialize them.

@@ -51,6 +51,8 @@ SIGNATURES = {
     "nvfp4_dequantize": ([_P, _P, _I, _P, _I64, _I64, _P, _I64, _P], _I),
     "nvfp4_gemm_workspace_bytes": ([_I64, _I64, _I64], _SZ),
     "nvfp4_gemm": ([_P, _P, _P, _I64, _P, _P, _P, _I64, _I64, _P, _I64, _P, _SZ, _P], _I),
+    "nvfp4_linear_workspace_bytes": ([_I64, _I64, _I64], _SZ),
+    "nvfp4_linear": ([_P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, _P, _I64, _P, _SZ, _P], _I),
     "nvfp4_read_device_error": ([_P, _P, ctypes.POINTER(ctypes.c_uint32)], _I),
     "nvfp4_last_launch_count": ([], _I),
     "nvfp4_quantize_noalloc": ([_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P, _P, _P], _I),
@@ -227,7 +229,25 @@ def last_launch_count() -> int:
     return load_library().nvfp4_last_launch_count()
 
 
-def linear(x: torch.Tensor, w: NVFP4Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """W4A4 linear layer: quantize the activation on the fly (absmax), then the GEMM."""
-    xq = nvfp4_quantize(x, "absmax", "swizzled", stream=stream)
-    return nvfp4_gemm(xq, w, out=out, stream=stream)
+def linear(x: torch.Tensor, w: NVFP4Tensor, x_global_scale: Optional[torch.Tensor] = None,
+           out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """W4A4 linear layer C = Q(x) w^T in BF16: the activation x (M x K BF16) is
+    quantized on this call with absmax block scales -- under `x_global_scale` (a
+    device float, e.g. a calibrated activation scale) or, if None, amax(|x|)/2688
+    computed on the device -- and multiplied by the pre-quantized weight w (N x K)."""
+    lib = load_library()
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D row-major bfloat16 CUDA tensor")
+    if w.layout != SF_SWIZZLED or w.cols != x.shape[1]:
+        raise ValueError("w must share K with x and have swizzled scales")
+    M, K = x.shape
+    N = w.rows
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(lib.nvfp4_linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=x.device)
+    st = lib.nvfp4_linear(_ptr(x), M, K, x.stride(0), _ptr(x_global_scale), _ptr(w.codes), _ptr(w.scales),
+                          _ptr(w.global_scale), N, _ptr(out), out.stride(0), _ptr(workspace), workspace.numel(),
+                          _stream(stream))
+    _check(st, "nvfp4_linear")
+    return out

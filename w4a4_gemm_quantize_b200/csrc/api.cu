@@ -36,6 +36,15 @@ nvfp4_status check_device_cached() {
 
 nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
+// Workspace of nvfp4_linear: [0, 256) the GEMM status word, [256, 260) the
+// activation's amax word, [260, 264) its global scale (large-M path), then from
+// byte 512 either the small-M kernel's counters and partial tiles or the
+// activation's codes (rounded up to 256 bytes) and swizzled scales.
+constexpr size_t kLinearHeader = 512;
+
+size_t linear_codes_bytes(int64_t M, int64_t K) { return (static_cast<size_t>(M) * (K / 2) + 255) / 256 * 256; }
+
+
 }  // namespace
 
 extern "C" {
@@ -72,31 +81,44 @@ size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout) {
 
 size_t nvfp4_quantize_workspace_bytes(int64_t, int64_t) { return kQuantizeWorkspace; }
 
-nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld_x, nvfp4_scale_mode mode,
-                            nvfp4_sf_layout layout, const float* global_scale_in, uint8_t* codes, uint8_t* scales,
-                            float* global_scale_out, float* block_err, void* workspace, size_t workspace_bytes,
-                            void* stream) {
-  nvfp4::g_last_launches = 0;
+}  // extern "C"
+
+namespace nvfp4 {
+
+nvfp4_status validate_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int mode, int layout,
+                               const float* global_scale_in, const uint8_t* codes, const uint8_t* scales,
+                               const float* global_scale_out, const float* block_err) {
   if (rows < 0 || cols < 0 || ld_x < cols) return NVFP4_ERR_INVALID_ARG;
   if (mode != NVFP4_SCALE_ABSMAX && mode != NVFP4_SCALE_MSE && mode != NVFP4_SCALE_FOUR_OVER_SIX)
     return NVFP4_ERR_INVALID_ARG;
   if (layout != NVFP4_SF_SWIZZLED && layout != NVFP4_SF_LINEAR) return NVFP4_ERR_INVALID_ARG;
   if (cols % 16 != 0) return NVFP4_ERR_SHAPE;
-  if (rows == 0 || cols == 0) {
-    if (global_scale_in == nullptr && (workspace == nullptr || workspace_bytes < kQuantizeWorkspace))
-      return NVFP4_ERR_WORKSPACE;
-  }
   if (rows > 0 && cols > 0 && (x == nullptr || codes == nullptr || scales == nullptr)) return NVFP4_ERR_INVALID_ARG;
-  if (global_scale_in == nullptr && (workspace == nullptr || workspace_bytes < kQuantizeWorkspace))
-    return NVFP4_ERR_WORKSPACE;
-  if ((x && !aligned16(x)) || (codes && !aligned16(codes)) || (scales && !aligned16(scales)) ||
-      (workspace && !aligned16(workspace)) || ld_x % 8 != 0)
+  if ((x && !aligned16(x)) || (codes && !aligned16(codes)) || (scales && !aligned16(scales)) || ld_x % 8 != 0)
     return NVFP4_ERR_ALIGNMENT;
   if ((global_scale_in && (reinterpret_cast<uintptr_t>(global_scale_in) & 3u)) ||
       (global_scale_out && (reinterpret_cast<uintptr_t>(global_scale_out) & 3u)) ||
       (block_err && (reinterpret_cast<uintptr_t>(block_err) & 3u)))
     return NVFP4_ERR_ALIGNMENT;
-  nvfp4_status st = check_device_cached();
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4
+
+extern "C" {
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld_x, nvfp4_scale_mode mode,
+                            nvfp4_sf_layout layout, const float* global_scale_in, uint8_t* codes, uint8_t* scales,
+                            float* global_scale_out, float* block_err, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  nvfp4::g_last_launches = 0;
+  nvfp4_status st = nvfp4::validate_quantize(x, rows, cols, ld_x, mode, layout, global_scale_in, codes, scales,
+                                             global_scale_out, block_err);
+  if (st != NVFP4_OK) return st;
+  if (global_scale_in == nullptr && (workspace == nullptr || workspace_bytes < kQuantizeWorkspace))
+    return NVFP4_ERR_WORKSPACE;
+  if (workspace && !aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+  st = check_device_cached();
   if (st != NVFP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -181,6 +203,60 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const f
                                            N, K, static_cast<uint16_t*>(c), ldc, status, s);
   if (e == cudaErrorInvalidValue) return NVFP4_ERR_CUDA;
   st = from_cuda(e);
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
+}
+
+size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 1) return kLinearHeader;
+  if (M <= 32) return kLinearHeader + nvfp4::gemm_scratch_bytes(M, N, K);
+  return kLinearHeader + linear_codes_bytes(M, K) + nvfp4_scales_bytes(M, K, NVFP4_SF_SWIZZLED);
+}
+
+nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, int64_t ld_x, const float* x_global_scale,
+                          const uint8_t* w_codes, const uint8_t* w_scales, const float* w_global_scale, int64_t N,
+                          void* c, int64_t ldc, void* workspace, size_t workspace_bytes, void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (M < 1 || N < 1 || K < 1 || ld_x < K || ldc < N) return NVFP4_ERR_INVALID_ARG;
+  if (K % 32 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return NVFP4_ERR_SHAPE;
+  if (!x || !w_codes || !w_scales || !w_global_scale || !c) return NVFP4_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < nvfp4_linear_workspace_bytes(M, N, K)) return NVFP4_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(c) || !aligned16(workspace) ||
+      ld_x % 8 != 0 || ldc % 8 != 0 || (reinterpret_cast<uintptr_t>(w_global_scale) & 3u) ||
+      (x_global_scale && (reinterpret_cast<uintptr_t>(x_global_scale) & 3u)))
+    return NVFP4_ERR_ALIGNMENT;
+  nvfp4_status st = check_device_cached();
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  uint32_t* amax_word = reinterpret_cast<uint32_t*>(ws + 256);
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  // one memset: the status word, the amax word and (small M) the tile counters
+  const size_t zero = M <= 32 ? kLinearHeader + (nvfp4::gemm_zero_bytes(M, N, K) - 256) : kLinearHeader;
+  if (cudaMemsetAsync(ws, 0, zero, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (x_global_scale == nullptr) {
+    st = from_cuda(nvfp4::launch_amax(xb, M, K, ld_x, amax_word, s));
+    if (st != NVFP4_OK) return st;
+    ++nvfp4::g_last_launches;
+  }
+  if (M <= 32) {
+    const cudaError_t e = nvfp4::launch_decode_quantize_x(
+        xb, M, K, ld_x, x_global_scale, x_global_scale ? nullptr : amax_word, w_codes, w_scales, w_global_scale, N,
+        static_cast<uint16_t*>(c), ldc, status, ws + kLinearHeader, s);
+    st = from_cuda(e);
+    if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+    return st;
+  }
+  uint8_t* a_codes = ws + kLinearHeader;
+  uint8_t* a_scales = a_codes + linear_codes_bytes(M, K);
+  float* a_gs = x_global_scale ? nullptr : reinterpret_cast<float*>(ws + 260);
+  st = from_cuda(nvfp4::launch_quantize(xb, M, K, ld_x, NVFP4_SCALE_ABSMAX, true, x_global_scale, amax_word, a_codes,
+                                        a_scales, a_gs, nullptr, s));
+  if (st != NVFP4_OK) return st;
+  ++nvfp4::g_last_launches;
+  st = from_cuda(nvfp4::launch_gemm(a_codes, a_scales, x_global_scale ? x_global_scale : a_gs, M, w_codes, w_scales,
+                                    w_global_scale, N, K, static_cast<uint16_t*>(c), ldc, status, s));
   if (st == NVFP4_OK) ++nvfp4::g_last_launches;
   return st;
 }

@@ -36,6 +36,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_block.cuh"
 
 namespace nvfp4 {
 
@@ -156,10 +157,9 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // The set-up above overlaps the previous kernel's tail (programmatic launch);
-  // from here on the operands it wrote are visible.  The status word is cleared
-  // here, long before any bounded wait could give up.
+  // from here on the operands it wrote are visible.  (The status word was cleared
+  // by a memset before the launch, so no CTA can erase another's timeout code.)
   grid_dependency_wait();
-  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
 
   if (warp == Cfg::PRODUCER_WARP) {
     if (lane == 0) {
@@ -445,8 +445,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // set-up overlapped the previous kernel's tail; its outputs are visible from here
+  // (the status word was cleared by a memset before the launch)
   grid_dependency_wait();
-  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
 
   if (warp == Cfg::PRODUCER_WARP) {
     if (lane == 0) {
@@ -716,23 +716,40 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 //
 // For a handful of activation rows the GEMM is a stream over the weights, so the
 // weight matrix B takes the MMA's 128-row A slot (D^T = B A^T, 128 x 32 x 64 per
-// instruction).  The stream is split evenly over the CTAs (one per SM): the K-tiles
-// of all 128-row weight tiles form one sequence of units, tile-major, and CTA c
-// takes units [c U / G, (c+1) U / G).  Every SM therefore streams the same number
-// of weight bytes, whatever the number of tiles.  A CTA's range can cross tile
-// boundaries; its part of one tile is a "segment" with its own accumulator, and
-// TMEM holds two accumulators so that the MMAs of a segment overlap the epilogue
-// of the one before.  A segment that covers a whole tile writes C.  Otherwise it
-// stores its FP32 partial tile; the segment of the tile that finishes last (atomic
-// counter) sums the tile's partials in segment order -- the result does not
-// depend on arrival order -- applies s_gA s_gB and writes C (transposed back) in
-// BF16, then clears the counter for the next call.
+// instruction).  The stream is split evenly over the CTAs: the K-tiles of all
+// 128-row weight tiles form one sequence of units, tile-major, and CTA c takes units
+// [c U / G, (c+1) U / G).  When the tiles number between 70 % and 100 % of the SMs,
+// G is the tile count and every CTA takes one whole tile; otherwise G is the SM
+// count and every SM streams the same number of weight bytes whatever the number of
+// tiles.  A CTA's range can cross tile boundaries; its part of one tile is a
+// "segment" with its own accumulator, and TMEM holds two accumulators so that the
+// MMAs of a segment overlap the epilogue of the one before.  A CTA works through its
+// partial segments first and its whole tiles last, so that the reductions of the
+// partial tiles overlap the streaming instead of trailing it.  A segment that
+// covers a whole tile writes C.  Otherwise it stores its FP32 partial tile; the
+// segment of the tile that finishes last (atomic counter) sums the tile's partials
+// in segment order -- the result does not depend on arrival order -- applies
+// s_gA s_gB and writes C (transposed back) in BF16, then clears the counter for
+// the next call.
 //
-// Scale factors reach TMEM through four "scale warps" (tcgen05.st of each lane's
-// 16-byte atom lines into a per-stage region, as in the pair kernel), not through
+// Scale factors reach TMEM through "scale warps" (tcgen05.st of each lane's 16-byte
+// atom lines into a per-stage region, as in the pair kernel), not through
 // tcgen05.cp: two copies per 128 x 32 x 64 MMA made the in-order tensor pipe, not
 // HBM, the limit.  The MMA issuer waits on one barrier per K-tile.
+//
+// QX (the activation quantized inside the GEMM, "NVFP4 en difusión ...", section 2:
+// the activation is quantized on every call, per 16-block, absmax): instead of
+// loading the activation's codes and scales, the scale warps quantize its BF16
+// K-tile themselves.  Two groups of four warps take alternate K-tiles; in a group,
+// warp q encodes K-quarter q (four blocks of each row) of the rows that exist (rows
+// past M stay zero), reading the values from global memory (the activation is at
+// most 32 rows and stays in L2) one K-tile ahead, writes the codes into the stage's
+// B tile in the MMA's K-major 128-byte-swizzled layout and the scale bytes into a
+// small per-stage array, gathers the group's scale words on an mbarrier, and then
+// moves the stage's scales to TMEM.  The arithmetic is the quantizer's absmax path,
+// operation for operation.
 
+template <bool QX>
 struct DecodeCfg {
   static constexpr int BM = 128;                 // weight rows per tile
   static constexpr int BN = 32;                  // activation rows (padded)
@@ -741,12 +758,15 @@ struct DecodeCfg {
   static constexpr int B_BYTES = BN * KTILE_BYTES;   // 4 KB of activation codes
   static constexpr int SF_ATOM = 512;
   static constexpr int SFA_BYTES = 4 * SF_ATOM;
-  static constexpr int SFB_BYTES = 4 * SF_ATOM;
+  // activation scales: 4 loaded atoms, or (QX) one 32-bit word per row and atom
+  static constexpr int SFB_BYTES = QX ? 4 * BN * 4 : 4 * SF_ATOM;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = 8;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
-  static constexpr int THREADS = 320;            // warps 0-3 epilogue, 4 producer, 5 MMA, 6-9 scales
+  static constexpr int TABLE_BYTES = QX ? static_cast<int>(sizeof(ScaleTables)) : 0;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + TABLE_BYTES + 512;
   static constexpr int SF_WARP0 = 6;
+  static constexpr int SF_GROUPS = QX ? 2 : 1;   // groups of four scale (quantizer) warps
+  static constexpr int THREADS = (SF_WARP0 + 4 * SF_GROUPS) * 32;  // 0-3 epilogue, 4 producer, 5 MMA
   static constexpr int TMEM_ACC = 0;             // two accumulators of 32 columns
   static constexpr int TMEM_SF = 64;             // one scale region of 32 columns per stage
   static constexpr int TMEM_COLS = 512;
@@ -772,25 +792,75 @@ __host__ __device__ inline int64_t decode_max_segments(int64_t KT, int64_t U, in
   return s < KT ? s : KT;
 }
 
-__global__ void __launch_bounds__(DecodeCfg::THREADS)
+// Segment k of a CTA's unit range [u0, u1) in processing order -- the partial
+// segments first (the head of the last tile, then the tail of the first), then the
+// whole tiles in order.  Returns false when the range has fewer segments.
+__device__ __forceinline__ bool decode_segment(int k, int64_t u0, int64_t u1, int64_t KT, int64_t& s0,
+                                               int64_t& s1) {
+  if (u0 >= u1) return false;
+  const int64_t t0 = u0 / KT, t1 = (u1 - 1) / KT;
+  if (t0 == t1) {
+    s0 = u0;
+    s1 = u1;
+    return k == 0;
+  }
+  const bool first_whole = (u0 % KT) == 0, last_whole = (u1 % KT) == 0;
+  int np = 0;
+  if (!last_whole) {
+    if (k == np) {
+      s0 = t1 * KT;
+      s1 = u1;
+      return true;
+    }
+    ++np;
+  }
+  if (!first_whole) {
+    if (k == np) {
+      s0 = u0;
+      s1 = (t0 + 1) * KT;
+      return true;
+    }
+    ++np;
+  }
+  const int64_t w0 = first_whole ? t0 : t0 + 1, w1 = last_whole ? t1 : t1 - 1;  // whole tiles [w0, w1]
+  const int64_t t = w0 + (k - np);
+  if (t > w1) return false;
+  s0 = t * KT;
+  s1 = s0 + KT;
+  return true;
+}
+
+// The activation's global scale inside a QX launch: the caller's, or RN32(amax / 2688)
+// from the amax pass (1 for an all-zero activation) -- the quantizer's rule.
+__device__ __forceinline__ float decode_x_scale(const float* x_gs_in, const uint32_t* x_amax) {
+  return global_scale(x_gs_in, x_amax);
+}
+
+template <bool QX>
+__global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                        const uint8_t* __restrict__ sf_w, const uint8_t* __restrict__ sf_x,
-                       const float* __restrict__ a_gs, const float* __restrict__ b_gs, uint16_t* __restrict__ C,
-                       int M, int N, int K, int64_t ldc, int max_seg, float* __restrict__ partial,
-                       uint32_t* __restrict__ counters, uint32_t* __restrict__ status) {
-  using Cfg = DecodeCfg;
+                       const float* __restrict__ a_gs, const float* __restrict__ b_gs,
+                       const uint16_t* __restrict__ xq, int64_t ld_x, const float* __restrict__ x_gs_in,
+                       const uint32_t* __restrict__ x_amax, uint16_t* __restrict__ C, int M, int N, int K,
+                       int64_t ldc, int max_seg, float* __restrict__ partial, uint32_t* __restrict__ counters,
+                       uint32_t* __restrict__ status) {
+  using Cfg = DecodeCfg<QX>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // every 128-byte-swizzled tile (A, B) starts on a 1024-byte boundary
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * Cfg::A_BYTES;
   uint8_t* sSFA = sB + STAGES * Cfg::B_BYTES;
   uint8_t* sSFB = sSFA + STAGES * Cfg::SFA_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * Cfg::SFB_BYTES);
+  ScaleTables* tab = reinterpret_cast<ScaleTables*>(sSFB + STAGES * Cfg::SFB_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * Cfg::SFB_BYTES + Cfg::TABLE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* sf_ready = empty + STAGES;
-  uint64_t* acc_full = sf_ready + STAGES;  // [2]
-  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint64_t* qdone = sf_ready + STAGES;     // [STAGES]: a quantizer group's scale words
+  uint64_t* acc_full = qdone + STAGES;     // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -809,7 +879,8 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&sf_ready[s], 4);  // lane 0 of each scale warp
+      mbar_init(&sf_ready[s], 4);  // lane 0 of each warp of the scale group
+      mbar_init(&qdone[s], 4);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -819,13 +890,22 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
     *abort_flag = 0u;
     fence_mbarrier_init();
   }
+  if (QX) {
+    // activation rows past M are never written: their codes and scale words stay zero
+    for (int i = threadIdx.x; i < STAGES * (Cfg::B_BYTES + Cfg::SFB_BYTES) / 16; i += blockDim.x) {
+      const int off = i * 16;
+      uint8_t* p = off < STAGES * Cfg::B_BYTES ? sB + off : sSFB + (off - STAGES * Cfg::B_BYTES);
+      *reinterpret_cast<uint4*>(p) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
   if (warp == 5) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
   if (warp == 4 && lane == 0) {
     prefetch_tmap(&tmap_w);
-    prefetch_tmap(&tmap_x);
+    if (!QX) prefetch_tmap(&tmap_x);
   }
   tc_fence_before();
   __syncthreads();
@@ -841,39 +921,50 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
       int64_t issued_last[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
-      for (int64_t u = u0, i = 0; u < u1; ++u, ++i) {
-        const int s = static_cast<int>(i % STAGES);
-        if (!mbar_wait(&empty[s], (static_cast<uint32_t>(i / STAGES) & 1u) ^ 1u, abort_flag, status, kErrWaitEmpty))
-          break;
-        const int tile = static_cast<int>(u / KT), kt = static_cast<int>(u - tile * KT);
-        const int ka0 = kt * 4;
-        const int na = min(4, k_atoms - ka0);
-        const uint32_t sf_bytes = static_cast<uint32_t>(na) * Cfg::SF_ATOM;
-        mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + 2 * sf_bytes);
-        tma_load_2d(sA + s * Cfg::A_BYTES, &tmap_w, &full[s], kt * Cfg::KTILE_BYTES, tile * Cfg::BM);
-        tma_load_2d(sB + s * Cfg::B_BYTES, &tmap_x, &full[s], kt * Cfg::KTILE_BYTES, 0);
-        bulk_load(sSFA + s * Cfg::SFA_BYTES, sf_w + (static_cast<size_t>(tile) * k_atoms + ka0) * Cfg::SF_ATOM,
-                  sf_bytes, &full[s]);
-        bulk_load(sSFB + s * Cfg::SFB_BYTES, sf_x + static_cast<size_t>(ka0) * Cfg::SF_ATOM, sf_bytes, &full[s]);
-        issued_last[s] = i;
+      int64_t i = 0, s0, s1;
+      bool ok = true;
+      for (int sg = 0; ok && decode_segment(sg, u0, u1, KT, s0, s1); ++sg) {
+        for (int64_t u = s0; u < s1; ++u, ++i) {
+          const int s = static_cast<int>(i % STAGES);
+          if (!mbar_wait(&empty[s], (static_cast<uint32_t>(i / STAGES) & 1u) ^ 1u, abort_flag, status,
+                         kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          const int tile = static_cast<int>(u / KT), kt = static_cast<int>(u - tile * KT);
+          const int ka0 = kt * 4;
+          const int na = min(4, k_atoms - ka0);
+          const uint32_t sf_bytes = static_cast<uint32_t>(na) * Cfg::SF_ATOM;
+          if constexpr (QX) {
+            mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + sf_bytes);
+          } else {
+            mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + 2 * sf_bytes);
+          }
+          tma_load_2d(sA + s * Cfg::A_BYTES, &tmap_w, &full[s], kt * Cfg::KTILE_BYTES, tile * Cfg::BM);
+          bulk_load(sSFA + s * Cfg::SFA_BYTES, sf_w + (static_cast<size_t>(tile) * k_atoms + ka0) * Cfg::SF_ATOM,
+                    sf_bytes, &full[s]);
+          if constexpr (!QX) {
+            tma_load_2d(sB + s * Cfg::B_BYTES, &tmap_x, &full[s], kt * Cfg::KTILE_BYTES, 0);
+            bulk_load(sSFB + s * Cfg::SFB_BYTES, sf_x + static_cast<size_t>(ka0) * Cfg::SF_ATOM, sf_bytes, &full[s]);
+          }
+          issued_last[s] = i;
+        }
       }
-      if (*abort_flag)
+      if (*abort_flag) {
         for (int s = 0; s < STAGES; ++s)
           if (issued_last[s] >= 0)
             mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_last[s] / STAGES) & 1u, status);
+      }
     }
   } else if (warp == 5) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
       const uint32_t idesc = idesc_mxf4nvf4(Cfg::BM, Cfg::BN);
       bool ok = true;
-      int q = 0;  // segment counter of this CTA
-      for (int64_t u = u0, i = 0; u < u1 && ok; ++u, ++i) {
-        const int tile = static_cast<int>(u / KT), kt = static_cast<int>(u - tile * KT);
-        const bool seg_first = (u == u0) || kt == 0;
-        const bool seg_last = (u + 1 == u1) || kt + 1 == KT;
+      int64_t i = 0, s0, s1;
+      for (int q = 0; ok && decode_segment(q, u0, u1, KT, s0, s1); ++q) {
         const int buf = q & 1;
-        if (seg_first && q >= 2) {
+        if (q >= 2) {
           if (!mbar_wait(&acc_empty[buf], static_cast<uint32_t>((q >> 1) - 1) & 1u, abort_flag, status,
                          kErrWaitAccEmpty)) {
             ok = false;
@@ -881,26 +972,27 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
           }
           tc_fence_after();
         }
-        const int s = static_cast<int>(i % STAGES);
-        // the scale warps arrive only after the stage's bytes landed and its scales are in TMEM
-        if (!mbar_wait(&sf_ready[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int na = min(4, k_atoms - kt * 4);
-        const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
-        const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
-        const uint32_t t_sf = tmem_base + Cfg::TMEM_SF + static_cast<uint32_t>(s) * 32;
         const uint32_t t_acc = tmem_base + Cfg::TMEM_ACC + buf * Cfg::BN;
-        for (int j = 0; j < na; ++j)
-          mma_mxf4nvf4(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
-                       t_sf + 4 * j, t_sf + 16 + 4 * j, (!seg_first || j != 0) ? 1u : 0u);
-        tc_commit(&empty[s]);
-        if (seg_last) {
-          tc_commit(&acc_full[buf]);
-          ++q;
+        for (int64_t u = s0; u < s1; ++u, ++i) {
+          const int kt = static_cast<int>(u % KT);
+          const int s = static_cast<int>(i % STAGES);
+          // the scale warps arrive only after the stage's bytes landed and its scales are in TMEM
+          if (!mbar_wait(&sf_ready[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int na = min(4, k_atoms - kt * 4);
+          const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
+          const uint32_t t_sf = tmem_base + Cfg::TMEM_SF + static_cast<uint32_t>(s) * 32;
+          for (int j = 0; j < na; ++j)
+            mma_mxf4nvf4(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
+                         t_sf + 4 * j, t_sf + 16 + 4 * j, (u != s0 || j != 0) ? 1u : 0u);
+          tc_commit(&empty[s]);
         }
+        if (!ok) break;
+        tc_commit(&acc_full[buf]);
       }
       if (!ok) {
         tc_commit(drain);
@@ -914,41 +1006,177 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
     // region of stage s is free once the stage's bytes land again: the producer
     // reloads a stage only after the MMAs that read it have completed.
     const uint32_t quarter = static_cast<uint32_t>(warp & 3);
-    for (int64_t u = u0, i = 0; u < u1; ++u, ++i) {
-      const int s = static_cast<int>(i % STAGES);
-      if (!warp_wait(&full[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull + 2)) break;
-      tc_fence_after();
-      const uint8_t* fa = sSFA + s * Cfg::SFA_BYTES + lane * 16;
-      const uint8_t* fb = sSFB + s * Cfg::SFB_BYTES + lane * 16;
-      uint32_t v[32];
+    const int group = (warp - Cfg::SF_WARP0) >> 2;
+    float d6 = 0.0f;
+    if constexpr (QX) {
+      // the activation's per-tensor scale and the 127 decoded scales, as the quantizer builds them
+      const float sg = decode_x_scale(x_gs_in, x_amax);
+      d6 = __fmul_rn(6.0f, sg);
+      const int t = threadIdx.x - Cfg::SF_WARP0 * 32;
+      if (t < 128) {
+        const float eff = __fmul_rn(e4m3_to_float(static_cast<uint32_t>(t)), sg);
+        tab->eff[t] = eff;
+        tab->rcp[t] = eff == 0.0f ? 0.0f : __frcp_rn(eff);
+      }
+      asm volatile("bar.sync 2, %0;" ::"n"(4 * Cfg::SF_GROUPS * 32) : "memory");  // the table is complete
+    }
+    // QX work items of a unit for this warp: (row, block) = (it / 4, it % 4) of its
+    // K-quarter, it = lane + 32 j over the M rows that exist (at most 4 per lane)
+    const int items = QX ? M * 4 : 0;
+    uint4 xv[4][2];  // the next unit's values: item j, 16 BF16 values as two 16-byte halves
+    auto load_unit = [&](int64_t u) {
+      const int kt = static_cast<int>(u % KT);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint4 a4 = *reinterpret_cast<const uint4*>(fa + j * Cfg::SF_ATOM);
-        const uint4 b4 = *reinterpret_cast<const uint4*>(fb + j * Cfg::SF_ATOM);
-        v[4 * j] = a4.x;
-        v[4 * j + 1] = a4.y;
-        v[4 * j + 2] = a4.z;
-        v[4 * j + 3] = a4.w;
-        v[16 + 4 * j] = b4.x;
-        v[16 + 4 * j + 1] = b4.y;
-        v[16 + 4 * j + 2] = b4.z;
-        v[16 + 4 * j + 3] = b4.w;
+        const int it = lane + 32 * j;
+        const int row = it >> 2, blk = it & 3;
+        const int k0 = kt * 256 + static_cast<int>(quarter) * 64 + blk * 16;
+        if (it < items && k0 < K) {
+          const uint4* p = reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(row) * ld_x + k0);
+          xv[j][0] = __ldcg(p);
+          xv[j][1] = __ldcg(p + 1);
+        } else {
+          xv[j][0] = make_uint4(0u, 0u, 0u, 0u);
+          xv[j][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
-      tmem_st_32x32b_x32(tmem_base + (quarter * 32u << 16) + Cfg::TMEM_SF + static_cast<uint32_t>(s) * 32, v);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sf_ready[s]);
+    };
+    int64_t i = 0, s0, s1, next_u = -1;
+    if (QX) {
+      // the first unit of this group
+      int64_t a0, a1;
+      for (int sg = 0, ii = 0; decode_segment(sg, u0, u1, KT, a0, a1); ++sg) {
+        if (a1 - a0 + ii > group) {
+          next_u = a0 + (group - ii);
+          break;
+        }
+        ii += static_cast<int>(a1 - a0);
+      }
+      if (next_u >= 0) load_unit(next_u);
+    }
+    bool ok = true;
+    for (int sg = 0; ok && decode_segment(sg, u0, u1, KT, s0, s1); ++sg) {
+      for (int64_t u = s0; u < s1; ++u, ++i) {
+        if (static_cast<int>(i % Cfg::SF_GROUPS) != group) continue;
+        const int s = static_cast<int>(i % STAGES);
+        uint32_t v[32];
+        if constexpr (QX) {
+          uint4 cur[4][2];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            cur[j][0] = xv[j][0];
+            cur[j][1] = xv[j][1];
+          }
+          // prefetch this group's next unit (the one SF_GROUPS units later in processing order)
+          {
+            int64_t nu = -1, ii = 0, a0, a1;
+            for (int g2 = 0; decode_segment(g2, u0, u1, KT, a0, a1); ++g2) {
+              const int64_t want = i + Cfg::SF_GROUPS;
+              if (want < ii + (a1 - a0)) {
+                if (want >= ii) nu = a0 + (want - ii);
+                break;
+              }
+              ii += a1 - a0;
+            }
+            if (nu >= 0) load_unit(nu);
+          }
+          // the stage's weight bytes landed, so the MMAs that last read its B tile are done
+          if (!warp_wait(&full[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull + 2)) {
+            ok = false;
+            break;
+          }
+          uint32_t* words = reinterpret_cast<uint32_t*>(sSFB + s * Cfg::SFB_BYTES);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int it = lane + 32 * j;
+            uint32_t sb = 0;
+            if (32 * j < items) {  // warp-uniform: the warp has items in this round
+              const uint32_t wd[8] = {cur[j][0].x, cur[j][0].y, cur[j][0].z, cur[j][0].w,
+                                      cur[j][1].x, cur[j][1].y, cur[j][1].z, cur[j][1].w};
+              uint64_t x2[8];
+              uint32_t mb = 0;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                x2[k] = pack2(__uint_as_float(wd[k] << 16), __uint_as_float(wd[k] & 0xFFFF0000u));
+                mb = __vmaxu2(mb, wd[k] & 0x7FFF7FFFu);
+              }
+              const float amax_b = bf16_bits_to_float(max(mb & 0xFFFFu, mb >> 16));
+              sb = cvt_e4m3_satfinite(__fdiv_rn(amax_b, d6));
+              uint32_t c0, c1;
+              encode_codes(x2, tab->eff[sb], tab->rcp[sb], c0, c1);
+              const int row = it >> 2, blk = it & 3;
+              if (it < items) {
+                // K bytes [32 quarter + 8 blk, +8) of row `row` in the K-major 128-byte-swizzled
+                // B tile: 16-byte chunk 2 quarter + blk / 2, swizzled by the row
+                const int chunk = (2 * static_cast<int>(quarter) + (blk >> 1)) ^ (row & 7);
+                *reinterpret_cast<uint2*>(sB + s * Cfg::B_BYTES + row * 128 + chunk * 16 + (blk & 1) * 8) =
+                    make_uint2(c0, c1);
+              }
+              // the row's four scale bytes of this K-quarter come from lanes 4r .. 4r+3
+              const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sb, 1);
+              const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, sb, 2);
+              const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, sb, 3);
+              if (it < items && blk == 0) words[quarter * 32 + row] = sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            }
+          }
+          fence_proxy_async_smem();  // the codes are read by the MMA (async proxy)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&qdone[s]);
+          if (!warp_wait(&qdone[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull + 7)) {
+            ok = false;
+            break;
+          }
+          const uint8_t* fa = sSFA + s * Cfg::SFA_BYTES + lane * 16;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 a4 = *reinterpret_cast<const uint4*>(fa + j * Cfg::SF_ATOM);
+            v[4 * j] = a4.x;
+            v[4 * j + 1] = a4.y;
+            v[4 * j + 2] = a4.z;
+            v[4 * j + 3] = a4.w;
+            // the atom line of lane L holds rows L, L+32, L+64, L+96: only row L exists
+            v[16 + 4 * j] = words[j * 32 + lane];
+            v[16 + 4 * j + 1] = 0u;
+            v[16 + 4 * j + 2] = 0u;
+            v[16 + 4 * j + 3] = 0u;
+          }
+        } else {
+          if (!warp_wait(&full[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull + 2)) {
+            ok = false;
+            break;
+          }
+          const uint8_t* fa = sSFA + s * Cfg::SFA_BYTES + lane * 16;
+          const uint8_t* fb = sSFB + s * Cfg::SFB_BYTES + lane * 16;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 a4 = *reinterpret_cast<const uint4*>(fa + j * Cfg::SF_ATOM);
+            const uint4 b4 = *reinterpret_cast<const uint4*>(fb + j * Cfg::SF_ATOM);
+            v[4 * j] = a4.x;
+            v[4 * j + 1] = a4.y;
+            v[4 * j + 2] = a4.z;
+            v[4 * j + 3] = a4.w;
+            v[16 + 4 * j] = b4.x;
+            v[16 + 4 * j + 1] = b4.y;
+            v[16 + 4 * j + 2] = b4.z;
+            v[16 + 4 * j + 3] = b4.w;
+          }
+        }
+        tc_fence_after();
+        tmem_st_32x32b_x32(tmem_base + (quarter * 32u << 16) + Cfg::TMEM_SF + static_cast<uint32_t>(s) * 32, v);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_ready[s]);
+      }
     }
   } else {
     // ---------------- epilogue (warps 0-3): lane = weight row n, 32 columns = activation rows m ----------------
-    const float alpha = __fmul_rn(*a_gs, *b_gs);
-    int q = 0;
-    for (int64_t u = u0; u < u1; ++q) {
-      const int tile = static_cast<int>(u / KT);
+    const float alpha = QX ? __fmul_rn(decode_x_scale(x_gs_in, x_amax), *b_gs) : __fmul_rn(*a_gs, *b_gs);
+    int64_t s0, s1;
+    for (int q = 0; decode_segment(q, u0, u1, KT, s0, s1); ++q) {
+      const int tile = static_cast<int>(s0 / KT);
       const int64_t tile_end = (static_cast<int64_t>(tile) + 1) * KT;
-      const int64_t seg_end = tile_end < u1 ? tile_end : u1;  // this segment: units [u, seg_end)
-      const bool whole = (u == static_cast<int64_t>(tile) * KT) && seg_end == tile_end;
+      const bool whole = (s0 == static_cast<int64_t>(tile) * KT) && s1 == tile_end;
       const int buf = q & 1;
       const bool got = warp_wait(&acc_full[buf], static_cast<uint32_t>(q >> 1) & 1u, abort_flag, status,
                                  kErrWaitAccFull);
@@ -1015,7 +1243,6 @@ __global__ void __launch_bounds__(DecodeCfg::THREADS)
           if (threadIdx.x == 0) counters[tile] = 0u;  // ready for the next call
         }
       }
-      u = seg_end;
     }
   }
 
@@ -1160,30 +1387,37 @@ cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float
                             static_cast<int>(N), static_cast<int>(K), status);
 }
 
-// CTAs of the stream-K decode kernel: one per SM, at most one per unit.
+// CTAs of the decode kernel: one per weight tile when the tiles number between 70 %
+// and 100 % of the SMs (no partial tiles), otherwise one per SM (at most one per unit).
 int64_t decode_grid(int64_t N, int64_t K, int sms) {
-  const int64_t U = ((N + DecodeCfg::BM - 1) / DecodeCfg::BM) * ((K + 255) / 256);
+  const int64_t T = (N + DecodeCfg<false>::BM - 1) / DecodeCfg<false>::BM;
+  const int64_t U = T * ((K + 255) / 256);
+  if (T <= sms && 10 * T >= 7 * static_cast<int64_t>(sms)) return T;  // one whole tile per CTA
   return U < sms ? U : sms;
 }
 
-cudaError_t launch_decode(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
-                          const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
-                          uint16_t* c, int64_t ldc, uint32_t* status, uint8_t* scratch, cudaStream_t stream) {
-  CUtensorMap tw, tx;
-  if (!encode_codes_map(&tw, b_codes, N, K, 128) || !encode_codes_map(&tx, a_codes, M, K, DecodeCfg::BN))
-    return cudaErrorInvalidValue;
+// Launch the decode kernel: QX = false reads the activation's codes and scales
+// (tmap_x over a_codes, a_sf, a_gs); QX = true quantizes the BF16 activation x (row
+// stride ld_x) itself, global scale from x_gs_in or the amax word x_amax.
+template <bool QX>
+cudaError_t launch_decode(const CUtensorMap& tw, const CUtensorMap& tx, const uint8_t* a_sf, const float* a_gs,
+                          const uint16_t* x, int64_t ld_x, const float* x_gs_in, const uint32_t* x_amax, int64_t M,
+                          const uint8_t* b_sf,
+                          const float* b_gs, int64_t N, int64_t K, uint16_t* c, int64_t ldc, uint32_t* status,
+                          uint8_t* scratch, cudaStream_t stream) {
+  using Cfg = DecodeCfg<QX>;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   static std::once_flag once[64];
-  cudaError_t attr_err = cudaSuccess;
+  static cudaError_t attr_err[64];
   std::call_once(once[dev & 63], [&] {
-    attr_err = cudaFuncSetAttribute(gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    DecodeCfg::SMEM_BYTES);
+    attr_err[dev & 63] = cudaFuncSetAttribute(gemm_decode_kernel<QX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              Cfg::SMEM_BYTES);
   });
-  if (attr_err != cudaSuccess) return attr_err;
+  if (attr_err[dev & 63] != cudaSuccess) return attr_err[dev & 63];
   const int64_t KT = (K + 255) / 256;
-  const int64_t U = ((N + DecodeCfg::BM - 1) / DecodeCfg::BM) * KT;
+  const int64_t U = ((N + Cfg::BM - 1) / Cfg::BM) * KT;
   const int64_t G = decode_grid(N, K, sms > kMaxDecodeGrid ? kMaxDecodeGrid : sms);
   const int max_seg = static_cast<int>(decode_max_segments(KT, U, G));
   // the counters were cleared together with the status word (gemm_zero_bytes)
@@ -1191,15 +1425,16 @@ cudaError_t launch_decode(const uint8_t* a_codes, const uint8_t* a_sf, const flo
   float* partial = reinterpret_cast<float*>(scratch + decode_counter_bytes(N));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(G));
-  cfg.blockDim = dim3(DecodeCfg::THREADS);
-  cfg.dynamicSmemBytes = DecodeCfg::SMEM_BYTES;
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   set_programmatic(attr[0]);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_decode_kernel, tw, tx, b_sf, a_sf, a_gs, b_gs, c, static_cast<int>(M),
-                            static_cast<int>(N), static_cast<int>(K), ldc, max_seg, partial, counters, status);
+  return cudaLaunchKernelEx(&cfg, gemm_decode_kernel<QX>, tw, tx, b_sf, a_sf, a_gs, b_gs, x, ld_x, x_gs_in, x_amax,
+                            c, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), ldc, max_seg, partial,
+                            counters, status);
 }
 
 template <int BN>
@@ -1208,13 +1443,16 @@ cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint
                         int64_t ldc, uint32_t* status, cudaStream_t stream) {
   using Cfg = GemmCfg<BN>;
   static std::once_flag once[64];
+  static cudaError_t attr_err[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  cudaError_t attr_err = cudaSuccess;
+  // the attribute is set once per device; its result is kept, so a failure is
+  // reported on every call, not only the first
   std::call_once(once[dev & 63], [&] {
-    attr_err = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+    attr_err[dev & 63] =
+        cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   });
-  if (attr_err != cudaSuccess) return attr_err;
+  if (attr_err[dev & 63] != cudaSuccess) return attr_err[dev & 63];
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + BN - 1) / BN);
@@ -1235,27 +1473,32 @@ cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint
 }  // namespace
 
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
-  if (M > DecodeCfg::BN) return 0;
+  using Cfg = DecodeCfg<false>;
+  if (M > Cfg::BN) return 0;
   // partial-tile slots for the largest grid the launcher uses (more CTAs, more segments)
   const int64_t KT = (K + 255) / 256;
-  const int64_t T = (N + DecodeCfg::BM - 1) / DecodeCfg::BM;
+  const int64_t T = (N + Cfg::BM - 1) / Cfg::BM;
   const int64_t G = decode_grid(N, K, kMaxDecodeGrid);
   const int64_t max_seg = decode_max_segments(KT, T * KT, G);
-  return decode_counter_bytes(N) + static_cast<size_t>(T * max_seg) * DecodeCfg::BM * DecodeCfg::BN * 4;
+  return decode_counter_bytes(N) + static_cast<size_t>(T * max_seg) * Cfg::BM * Cfg::BN * 4;
 }
 
 size_t gemm_zero_bytes(int64_t M, int64_t N, int64_t) {
-  // the decode kernel's status word and tile counters; the tile kernels clear their
-  // status word themselves, so nothing separates them from the kernel before them
-  return M <= DecodeCfg::BN ? 256 + decode_counter_bytes(N) : 0;
+  // the status word of every kernel (a clear inside the kernel could erase the
+  // timeout code of a CTA that started earlier), plus the decode kernel's tile counters
+  return M <= DecodeCfg<false>::BN ? 256 + decode_counter_bytes(N) : sizeof(uint32_t);
 }
 
 cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
                         uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream) {
-  if (M <= DecodeCfg::BN)
-    return launch_decode(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status,
-                         reinterpret_cast<uint8_t*>(status) + 256, stream);
+  if (M <= DecodeCfg<false>::BN) {
+    CUtensorMap tw, tx;
+    if (!encode_codes_map(&tw, b_codes, N, K, 128) || !encode_codes_map(&tx, a_codes, M, K, DecodeCfg<false>::BN))
+      return cudaErrorInvalidValue;
+    return launch_decode<false>(tw, tx, a_sf, a_gs, nullptr, 0, nullptr, nullptr, M, b_sf, b_gs, N, K, c, ldc, status,
+                                reinterpret_cast<uint8_t*>(status) + 256, stream);
+  }
   if (M > 128 && N > 128)
     return launch_pair(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status, stream);
   const int bn = N > 128 ? 256 : 128;
@@ -1264,6 +1507,17 @@ cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
     return cudaErrorInvalidValue;
   if (bn == 256) return launch_tile<256>(ta, tb, a_sf, b_sf, a_gs, b_gs, M, N, K, c, ldc, status, stream);
   return launch_tile<128>(ta, tb, a_sf, b_sf, a_gs, b_gs, M, N, K, c, ldc, status, stream);
+}
+
+cudaError_t launch_decode_quantize_x(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* x_gs_in,
+                                     const uint32_t* x_amax, const uint8_t* b_codes, const uint8_t* b_sf,
+                                     const float* b_gs, int64_t N, uint16_t* c, int64_t ldc, uint32_t* status,
+                                     uint8_t* scratch, cudaStream_t stream) {
+  CUtensorMap tw;
+  if (!encode_codes_map(&tw, b_codes, N, K, 128)) return cudaErrorInvalidValue;
+  // (the activation is read with plain loads; the second tensor-map slot is unused)
+  return launch_decode<true>(tw, tw, nullptr, nullptr, x, ld_x, x_gs_in, x_amax, M, b_sf, b_gs, N, K, c, ldc, status,
+                             scratch, stream);
 }
 
 }  // namespace nvfp4

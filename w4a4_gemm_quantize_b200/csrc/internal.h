@@ -5,7 +5,15 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "../../include/nvfp4.h"
+
 namespace nvfp4 {
+
+// Host-side checks of nvfp4_quantize's arguments other than the workspace (api.cu),
+// made before any CUDA call: NVFP4_OK or the status the entry point returns.
+nvfp4_status validate_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int mode, int layout,
+                               const float* global_scale_in, const uint8_t* codes, const uint8_t* scales,
+                               const float* global_scale_out, const float* block_err);
 
 // Quantizer launchers (quantize.cu).  All pointers are device pointers that the
 // API layer has already validated.
@@ -26,14 +34,22 @@ cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
                         uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream);
 
+// The small-M GEMM (M <= 32) that quantizes its BF16 activation x (M x K, row stride
+// ld_x) itself, absmax block scales under the global scale *x_gs_in, or, when x_gs_in
+// is null, RN32(amax / 2688) from the amax word x_amax written by launch_amax.
+// scratch: the decode kernel's counters (zeroed) and partial tiles.
+cudaError_t launch_decode_quantize_x(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* x_gs_in,
+                                     const uint32_t* x_amax, const uint8_t* b_codes, const uint8_t* b_sf,
+                                     const float* b_gs, int64_t N, uint16_t* c, int64_t ldc, uint32_t* status,
+                                     uint8_t* scratch, cudaStream_t stream);
+
 // Bytes the GEMM needs in its workspace after the 256-byte status block
 // (split-K partial tiles of the small-M kernel); 0 when none.
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 
-// Bytes at the start of the workspace that must be zero when the GEMM launches:
-// for M <= 32 the decode kernel's status word and its tile counters after the
-// 256-byte status block (cleared with one memset); 0 for the tile kernels, which
-// clear their status word themselves.
+// Bytes at the start of the workspace that must be zero when the GEMM launches
+// (cleared with one memset before the kernel): the status word, and for M <= 32
+// the decode kernel's tile counters after the 256-byte status block.
 size_t gemm_zero_bytes(int64_t M, int64_t N, int64_t K);
 
 // Number of kernel launches the last call of each entry point enqueued (for

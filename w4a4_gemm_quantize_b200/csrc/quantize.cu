@@ -33,6 +33,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_block.cuh"
 
 namespace nvfp4 {
 
@@ -57,8 +58,6 @@ __device__ __forceinline__ uint32_t vmax_mag(uint32_t m, uint4 v) {
   m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
   return m;
 }
-
-__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
 
 // Global amax: the largest |x| as the 15-bit magnitude pattern of a BF16 value
 // (for non-negative BF16 values the integer order of the bit patterns is the
@@ -102,99 +101,8 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
   }
 }
 
-// Two binary32 values in one 64-bit register (element 2i low, 2i+1 high) for the
-// packed f32x2 arithmetic of sm_100.
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-
-__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-
-// RN32(a * b) on both halves.
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-// RN32(a * b + c) on both halves (one rounding each).
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-
-// Sign bit of each of the 16 values moved to bit 3 of its code nibble.
-__device__ __forceinline__ void sign_codes(const uint64_t (&x2)[8], uint32_t& c0, uint32_t& c1) {
-  c0 = c1 = 0u;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = static_cast<uint32_t>(x2[i]) >> 31, hi = static_cast<uint32_t>(x2[i] >> 32) >> 31;
-    const uint32_t nib = (lo << 3) | (hi << 7);
-    if (i < 4)
-      c0 |= nib << (8 * i);
-    else
-      c1 |= nib << (8 * (i - 4));
-  }
-}
-
-// Signed 4-bit codes of 16 values (packed pairs x2) for effective scale eff with
-// rcp = RN32(1/eff): y = RN32(x * rcp) rounded to the E2M1 grid (RNE, saturating),
-// the sign of x kept by the conversion (-0 and small negatives give code 0x8).
-__device__ __forceinline__ void encode_codes(const uint64_t (&x2)[8], float eff, float rcp, uint32_t& c0,
-                                             uint32_t& c1) {
-  if (eff == 0.0f) {  // zero scale: every magnitude is 0, only the signs remain
-    sign_codes(x2, c0, c1);
-    return;
-  }
-  const uint64_t r2 = pack2(rcp, rcp);
-  float y[16];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) unpack2(mul2(x2[i], r2), y[2 * i], y[2 * i + 1]);
-  if (isinf(rcp)) {
-    // 1/eff overflowed: +-0 * inf is NaN; a zero input keeps its own (signed) zero
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float lo, hi;
-      unpack2(x2[i], lo, hi);
-      if (lo == 0.0f) y[2 * i] = lo;
-      if (hi == 0.0f) y[2 * i + 1] = hi;
-    }
-  }
-  c0 = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-  c1 = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
-}
-
-// Squared reconstruction error of the block in element order:
-// d_k = RN32(x_k - q_k * eff) (one fma), e = fma(d_k, d_k, e), k = 0..15.
-__device__ __forceinline__ float block_sse(const uint64_t (&x2)[8], uint32_t c0, uint32_t c1, float eff) {
-  const uint64_t neff2 = pack2(-eff, -eff);
-  float e = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t h2 = e2m1x2_to_half2(i < 4 ? c0 : c1, i & 3);
-    const float q_lo = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFFu)));
-    const float q_hi = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 >> 16)));
-    float d_lo, d_hi;
-    unpack2(fma2(pack2(q_lo, q_hi), neff2, x2[i]), d_lo, d_hi);
-    e = __fmaf_rn(d_lo, d_lo, e);
-    e = __fmaf_rn(d_hi, d_hi, e);
-  }
-  return e;
-}
-
 __device__ __forceinline__ int64_t swizzled_offset(int64_t r, int64_t c, int64_t atoms_per_group) {
   return ((r >> 7) * atoms_per_group + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
-}
-
-__device__ __forceinline__ float global_scale(const float* gs_in, const uint32_t* amax_bits) {
-  if (gs_in) return *gs_in;
-  const float amax = bf16_bits_to_float(*amax_bits);
-  return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
 
 // Zero the padding of a swizzled scale buffer (rows [rows, Rp) and block columns
@@ -222,15 +130,6 @@ __device__ __forceinline__ void zero_scale_padding(uint8_t* __restrict__ scales,
     scales[swizzled_offset(r, c, atoms_per_group)] = 0;
   }
 }
-
-// The 127 finite non-negative E4M3 scale bytes of one tensor, decoded: eff =
-// RN32(dec(s) s_g) and RN32(1/eff) (0 for eff = 0).  Every CTA builds them once, so
-// each candidate scale costs two shared-memory reads instead of a conversion, a
-// product and a correctly rounded reciprocal.
-struct ScaleTables {
-  float eff[128];
-  float rcp[128];
-};
 
 // One warp handles 32 consecutive blocks of one row (lane = block); warps walk a
 // fixed column chunk down the rows, so block coordinates and output offsets need
