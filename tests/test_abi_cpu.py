@@ -171,3 +171,22 @@ def test_bench_profile_record_matches_only_its_sources(tmp_path, monkeypatch):
     (tmp_path / "profiles" / "gemm_w.md").write_text("- source_hash: `0000000000000000`\n- traffic_bytes_per_launch: 1234\n")
     assert bench.profiled_traffic("gemm", "w") is None
     assert bench.profiled_traffic("gemm", "missing") is None
+
+
+def test_noalloc_validation_before_any_cuda_call(lib):
+    """The no-allocation quantizer checks its arguments on the host first, then the device
+    (without a GPU it reports the device), before it looks up its scratch block."""
+    P = ctypes.c_void_p
+
+    def q(x=16, rows=4, cols=32, ld=32, mode=0, layout=0, codes=16, scales=16):
+        return lib.nvfp4_quantize_noalloc(P(x) if x else None, rows, cols, ld, mode, layout, None,
+                                          P(codes) if codes else None, P(scales) if scales else None, None, None,
+                                          None)
+
+    assert q(cols=24, ld=24) == 2
+    assert q(rows=-1) == 1
+    assert q(mode=9) == 1
+    assert q(x=0) == 1
+    assert q(x=8) == 3
+    assert q(ld=36) == 3
+    assert q() in (4, 5)

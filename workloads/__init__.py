@@ -40,12 +40,35 @@ def to_bf16(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).contiguous()
 
 
-def normal(shape, seed: int, stream: int, std: float = 1.0) -> np.ndarray:
-    return (rng(seed, stream).standard_normal(size=shape, dtype=np.float32) * np.float32(std))
+def normal(shape, seed: int, stream: int, std: float = 1.0, chunk: int = 1 << 22) -> np.ndarray:
+    g = rng(seed, stream)
+    n = int(np.prod(shape))
+    out = np.empty(n, np.float32)
+    for i in range(0, n, chunk):
+        m = min(chunk, n - i)
+        out[i:i + m] = g.standard_normal(m, dtype=np.float32) * np.float32(std)
+    return out.reshape(shape)
 
 
-def student_t(shape, nu: int, scale: float, seed: int, stream: int) -> np.ndarray:
-    return (rng(seed, stream).standard_t(nu, size=shape) * scale).astype(np.float32)
+def student_t(shape, nu: int, scale: float, seed: int, stream: int, chunk: int = 1 << 22) -> np.ndarray:
+    """scale * Student-t(nu) for an integer nu, drawn as z / sqrt(chi2_nu / nu) with
+    z ~ N(0,1) and chi2_nu the sum of nu // 2 terms -2 ln(U) (U uniform on (0, 1]) plus
+    one squared normal when nu is odd -- an exact construction of the distribution,
+    generated in chunks of `chunk` values."""
+    g = rng(seed, stream)
+    n = int(np.prod(shape))
+    out = np.empty(n, np.float32)
+    for i in range(0, n, chunk):
+        m = min(chunk, n - i)
+        z = g.standard_normal(m, dtype=np.float32)
+        chi = np.zeros(m, np.float32)
+        for _ in range(nu // 2):
+            chi -= np.float32(2) * np.log1p(-g.random(m, dtype=np.float32))
+        if nu % 2:
+            chi += g.standard_normal(m, dtype=np.float32) ** 2
+        chi = np.maximum(chi, np.float32(1e-30))
+        out[i:i + m] = z / np.sqrt(chi / np.float32(nu)) * np.float32(scale)
+    return out.reshape(shape)
 
 
 def with_outlier_entries(a: np.ndarray, prob: float, factor: float, seed: int, stream: int) -> np.ndarray:
