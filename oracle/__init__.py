@@ -101,6 +101,14 @@ def _load():
     lib.ora_f32_to_bf16_array.restype = None
     lib.ora_lora_f64.argtypes = [P, I64, I64, P, I64, P, I64, P, P, P]
     lib.ora_lora_f64.restype = ctypes.c_int
+    lib.ora_e8m0_decode.argtypes = [ctypes.c_uint8]
+    lib.ora_e8m0_decode.restype = ctypes.c_double
+    lib.ora_quantize_mx.argtypes = [P, I64, I64, I64, P, P]
+    lib.ora_quantize_mx.restype = ctypes.c_int
+    lib.ora_dequantize_mx.argtypes = [P, P, I64, I64, P]
+    lib.ora_dequantize_mx.restype = None
+    lib.ora_gemm_mx_f64_at.argtypes = [P, P, P, P, I64, P, P, I64, P, P]
+    lib.ora_gemm_mx_f64_at.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -303,3 +311,56 @@ def unpack_codes(codes: np.ndarray) -> np.ndarray:
     out[:, 0::2] = codes & 0xF
     out[:, 1::2] = codes >> 4
     return out
+
+
+# --- MXFP4 (outside reading: the OCP Microscaling Formats specification v1.0) ----------------------
+
+def e8m0_decode(b: int) -> float:
+    """E8M0 scale byte b -> 2^(b - 127) (0xFF = NaN)."""
+    return _load().ora_e8m0_decode(b)
+
+
+def quantize_mx(x):
+    """MXFP4: blocks of 32 along the row, E8M0 scale 2^(floor(log2 amax) - 2), E2M1 elements.
+
+    Returns (codes uint8 [rows, cols/2], scales uint8 [rows, cols/32] linear E8M0)."""
+    x = _bits(x)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 32), np.uint8)
+    if _load().ora_quantize_mx(_ptr(x), rows, cols, cols, _ptr(codes), _ptr(scales)) != 0:
+        raise ValueError(f"bad shape {x.shape}")
+    return codes, scales
+
+
+def dequantize_mx(codes, scales) -> np.ndarray:
+    """BF16 bits of q * 2^(s - 127)."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    rows, half = codes.shape
+    out = np.empty((rows, half * 2), np.uint16)
+    _load().ora_dequantize_mx(_ptr(codes), _ptr(scales), rows, half * 2, _ptr(out))
+    return out
+
+
+def gemm_mx_f64_at(a_codes, a_scales, b_codes, b_scales, m_idx, n_idx):
+    """Binary64 C = A B^T of MXFP4 operands at positions (m_idx[i], n_idx[i]); returns (C, S)."""
+    a_codes, b_codes = np.ascontiguousarray(a_codes, np.uint8), np.ascontiguousarray(b_codes, np.uint8)
+    a_scales, b_scales = np.ascontiguousarray(a_scales, np.uint8), np.ascontiguousarray(b_scales, np.uint8)
+    m_idx = np.ascontiguousarray(m_idx, np.int64)
+    n_idx = np.ascontiguousarray(n_idx, np.int64)
+    out = np.empty(m_idx.shape, np.float64)
+    absum = np.empty(m_idx.shape, np.float64)
+    if _load().ora_gemm_mx_f64_at(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), a_codes.shape[1] * 2,
+                                  _ptr(m_idx), _ptr(n_idx), m_idx.size, _ptr(out), _ptr(absum)) != 0:
+        raise MemoryError("oracle GEMM work buffer")
+    return out, absum
+
+
+def gemm_mx_f64(a_codes, a_scales, b_codes, b_scales):
+    """Binary64 C = A B^T of MXFP4 operands, all positions; returns (C [M, N], S)."""
+    M, N = a_codes.shape[0], b_codes.shape[0]
+    mi = np.repeat(np.arange(M), N)
+    ni = np.tile(np.arange(N), M)
+    c, s = gemm_mx_f64_at(a_codes, a_scales, b_codes, b_scales, mi, ni)
+    return c.reshape(M, N), s.reshape(M, N)

@@ -526,3 +526,117 @@ int ora_lora_f64(const uint16_t *x, int64_t M, int64_t K, const uint16_t *a, int
     free(t);
     return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* MXFP4 (NEXT: the "MXFP4 / NVFP4: Blackwell agresivo" section of "Cuantización */
+/* en Producción: AWQ, GPTQ, GGUF K-quants, FP8, MXFP4/NVFP4" names the format  */
+/* but gives neither its block size nor its scale type).  Outside reading, the  */
+/* public OCP Microscaling Formats (MX) specification v1.0: blocks of 32 values  */
+/* along K, one E8M0 scale per block (a power of two 2^(e - 127), e = 0..254,    */
+/* 0xFF = NaN), E2M1 elements, no per-tensor scale.  The block's scale is       */
+/* 2^(floor(log2(amax)) - 2) -- 2 being the exponent of the largest E2M1 value   */
+/* 6 = 1.5 * 2^2 -- clamped to the E8M0 range; each element is x / 2^e rounded  */
+/* to the E2M1 grid (RNE, saturating at 6, the sign kept).  An all-zero block   */
+/* takes the smallest scale (byte 0).                                          */
+/* ------------------------------------------------------------------------- */
+
+double ora_e8m0_decode(uint8_t b)
+{
+    if (b == 0xFF)
+        return NAN;
+    return ldexp(1.0, (int)b - 127);
+}
+
+/* floor(log2(a)) of a positive finite float, exact (frexp: a = f 2^e, 0.5 <= f < 1). */
+static int floor_log2f(float a)
+{
+    int e;
+    frexpf(a, &e);
+    return e - 1;
+}
+
+/* One block of 32: returns the E8M0 scale byte; codes[k] gets the signed 4-bit code. */
+static uint8_t mx_quantize_block(const float x[32], uint8_t codes[32])
+{
+    float amax = 0.0f;
+    for (int k = 0; k < 32; k++) {
+        float a = fabsf(x[k]);
+        if (a > amax)
+            amax = a;
+    }
+    int shared = (amax == 0.0f) ? -127 : floor_log2f(amax) - 2;
+    if (shared < -127)
+        shared = -127;
+    if (shared > 127)
+        shared = 127;
+    for (int k = 0; k < 32; k++) {
+        /* |x| / 2^shared, exact in binary64 (8 significant bits); below binary32's range
+           the value is far below the smallest E2M1 step and codes to 0 either way */
+        float y = (float)ldexp((double)fabsf(x[k]), -shared);
+        uint8_t mag = (x[k] == 0.0f) ? 0 : ora_e2m1_encode_mag(y);
+        codes[k] = (uint8_t)((signbit(x[k]) ? 8 : 0) | mag);
+    }
+    return (uint8_t)(shared + 127);
+}
+
+/* x: rows x cols BF16 bits (row stride ld), cols % 32 == 0.  codes (rows, cols/2),
+   scales (rows, cols/32) linear.  Returns 0, or -1 on a bad shape. */
+int ora_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, uint8_t *codes, uint8_t *scales)
+{
+    if (rows < 0 || cols < 0 || cols % 32 != 0 || ld < cols)
+        return -1;
+    int64_t nblk = cols / 32;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t b = 0; b < nblk; b++) {
+            float xb[32];
+            uint8_t c[32];
+            for (int k = 0; k < 32; k++)
+                xb[k] = ora_bf16_to_f32(x[r * ld + b * 32 + k]);
+            scales[r * nblk + b] = mx_quantize_block(xb, c);
+            for (int j = 0; j < 16; j++)
+                codes[r * (cols / 2) + b * 16 + j] = (uint8_t)((c[2 * j] & 0xF) | (c[2 * j + 1] << 4));
+        }
+    return 0;
+}
+
+/* BF16 bits of q * 2^(s - 127) (exact in binary32, rounded to BF16 RNE). */
+void ora_dequantize_mx(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols, uint16_t *out)
+{
+    int64_t nblk = cols / 32;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++) {
+            uint8_t byte = codes[r * (cols / 2) + c / 2];
+            uint8_t code = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+            double v = ora_e2m1_decode(code) * ora_e8m0_decode(scales[r * nblk + c / 32]);
+            out[r * cols + c] = ora_f32_to_bf16((float)v);
+        }
+}
+
+/* Row of an MXFP4 operand as binary64 values q * 2^(s - 127) (each exact). */
+static void decode_row_mx(const uint8_t *codes, const uint8_t *scales, int64_t row, int64_t K, double *out)
+{
+    for (int64_t k = 0; k < K; k++) {
+        uint8_t byte = codes[row * (K / 2) + k / 2];
+        uint8_t code = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+        out[k] = ora_e2m1_decode(code) * ora_e8m0_decode(scales[row * (K / 32) + k / 32]);
+    }
+}
+
+/* C = A B^T of two MXFP4 operands (A M x K, B N x K, linear scales), binary64, with
+   absum = sum |a b|; at `count` sampled positions (m_idx[i], n_idx[i]). */
+int ora_gemm_mx_f64_at(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *b_codes,
+                       const uint8_t *b_scales, int64_t K, const int64_t *m_idx, const int64_t *n_idx, int64_t count,
+                       double *out, double *absum)
+{
+    double *a = (double *)malloc(sizeof(double) * (size_t)(2 * K));
+    if (!a)
+        return -1;
+    double *b = a + K;
+    for (int64_t i = 0; i < count; i++) {
+        decode_row_mx(a_codes, a_scales, m_idx[i], K, a);
+        decode_row_mx(b_codes, b_scales, n_idx[i], K, b);
+        dot_f64(a, b, K, &out[i], absum ? &absum[i] : NULL);
+    }
+    free(a);
+    return 0;
+}
