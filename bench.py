@@ -66,6 +66,10 @@ WORKLOADS = {
     "decode_m8": dict(kind="decode", M=8, N=14336, K=4096),
     "decode_m32": dict(kind="decode", M=32, N=14336, K=4096),
     "mse4096": dict(kind="mse", rows=4096, cols=4096),
+    "decode_m32_lora16": dict(kind="decode_lora", M=32, N=14336, K=4096, R=16),
+    "decode_m32_lora64": dict(kind="decode_lora", M=32, N=14336, K=4096, R=64),
+    "prefill8b_lora16": dict(kind="prefill_lora", M=4096, K_up=4096, N_up=14336, K_down=14336, N_down=4096, R=16),
+    "prefill8b_lora64": dict(kind="prefill_lora", M=4096, K_up=4096, N_up=14336, K_down=14336, N_down=4096, R=64),
     "pr1": dict(kind="pr1", M=16, N=256, K=256),
 }
 
@@ -243,6 +247,14 @@ def gemm_work(M, N, K):
     return {"flops": 2.0 * M * N * K, "bytes": (M + N) * K * 0.5625 + 2.0 * M * N}
 
 
+def lora_work(M, N, K, R):
+    """The low-rank linear layer's FLOPs (W4A4 GEMM plus both low-rank products) and
+    algorithmic bytes (weight codes and scales, X in BF16, the factors, t, C)."""
+    w = gemm_work(M, N, K)
+    return {"flops": w["flops"] + 2.0 * M * K * R + 2.0 * M * N * R,
+            "bytes": N * K * 0.5625 + M * K * 2.0 + (R * K + N * R) * 2.0 + 2.0 * M * N}
+
+
 def gemm_kernel_name(M: int, N: int) -> str:
     """The kernel the library picks for an M x N output (its launch dispatch)."""
     if M <= 32:
@@ -262,6 +274,14 @@ def host_inputs(cfg, seed: int, rank: int):
                 "W2": W.t4_weight(cfg["N2"], cfg["K2"], seed=s, stream=W.STREAM_W2),
                 "X": W.activation(cfg["M"], cfg["K1"], seed=s, stream=W.STREAM_X, n_outlier_channels=0),
                 "X2": W.activation(cfg["M"], cfg["K2"], seed=s, stream=W.STREAM_X2, n_outlier_channels=0)}
+    if k in ("prefill_lora", "decode_lora"):
+        base = host_inputs({**cfg, "kind": k.split("_")[0]}, seed, rank)
+        R = cfg["R"]
+        for suf, (n, kk) in ((("_up", (cfg["N_up"], cfg["K_up"])), ("_down", (cfg["N_down"], cfg["K_down"])))
+                             if k == "prefill_lora" else (("", (cfg["N"], cfg["K"])),)):
+            base["A" + suf] = W.to_bf16(W.normal((R, kk), s, 11, 0.02))
+            base["B" + suf] = W.to_bf16(W.normal((n, R), s, 12, 0.1))
+        return base
     if k == "prefill":
         return {"W_up": W.gaussian_weight(cfg["N_up"], cfg["K_up"], 0.02, seed=s, stream=W.STREAM_W),
                 "W_down": W.gaussian_weight(cfg["N_down"], cfg["K_down"], 0.02, seed=s, stream=W.STREAM_W2),
@@ -281,7 +301,7 @@ def host_inputs(cfg, seed: int, rank: int):
 # Each step's inputs copied from the host in the end-to-end measurement (weights that
 # the step only reads are resident model parameters), and the results read back.
 E2E_INPUTS = {"dense31b": ["W", "W2", "X", "X2"], "prefill": ["X_up", "X_down"], "decode": ["X"],
-              "mse": ["W"], "pr1": ["W", "X"]}
+              "mse": ["W"], "pr1": ["W", "X"], "prefill_lora": ["X_up", "X_down"], "decode_lora": ["X"]}
 
 
 def describe(cfg):
@@ -293,6 +313,10 @@ def describe(cfg):
         "decode": "C = Q(X) W^T in one kernel: X's absmax block scales computed on the fly under a calibrated "
                   "per-tensor scale (weight MSE-quantized once before timing)",
         "mse": "MSE-quantize W (8 candidate scales, global scale computed in the step)",
+        "decode_lora": f"C = Q(X) W^T + (X A^T) B^T, rank {cfg.get('R')}: the low-rank down-projection, then one "
+                       "kernel quantizing X and adding B t to the FP4 accumulator (calibrated activation scale)",
+        "prefill_lora": f"up and down projections with a rank-{cfg.get('R')} low-rank branch: down-projection, "
+                        "absmax quantization of X, CTA-pair GEMM with the low-rank MMAs (calibrated activation scale)",
         "pr1": "absmax-quantize W and X, C = X W^T",
     }[k]
 
@@ -341,6 +365,18 @@ class Replica:
         elif k == "mse":
             q["W"] = nv.nvfp4_quantize(self.x["W"], "mse", block_err=True)
             self._ws(device, [], ["W"])
+        elif k in ("decode_lora", "prefill_lora"):
+            lib = nv.load_library()
+            R = cfg["R"]
+            self.x_scale = {}
+            sufs = [("_up", cfg.get("N_up"), cfg.get("K_up")), ("_down", cfg.get("N_down"), cfg.get("K_down"))] \
+                if k == "prefill_lora" else [("", cfg["N"], cfg["K"])]
+            for suf, n, kk in sufs:
+                q["W" + suf] = nv.nvfp4_quantize(self.x["W" + suf], "mse")
+                self.x_scale[suf] = nv.nvfp4_quantize(self.x["X" + suf], "absmax").global_scale.clone()
+                self.out["C" + suf] = torch.empty((cfg["M"], n), dtype=torch.bfloat16, device=device)
+                self.ws["lin" + suf] = torch.empty(lib.nvfp4_linear_lora_workspace_bytes(cfg["M"], n, kk, R),
+                                                   dtype=torch.uint8, device=device)
         elif k == "pr1":
             q["W"] = nv.nvfp4_quantize(self.x["W"], "absmax")
             q["X"] = nv.nvfp4_quantize(self.x["X"], "absmax")
@@ -366,6 +402,12 @@ class Replica:
     def _quant(self, name, mode):
         nv = self.nv
         return lambda: nv.nvfp4_quantize(self.x[name], mode, out=self.q[name], workspace=self.ws[name])
+
+    def _lora(self, suf):
+        nv = self.nv
+        return lambda: nv.linear_lora(self.x["X" + suf], self.q["W" + suf], self.x["A" + suf], self.x["B" + suf],
+                                      x_global_scale=self.x_scale[suf], out=self.out["C" + suf],
+                                      workspace=self.ws["lin" + suf])
 
     def _gemm(self, a, b, c, ws):
         nv = self.nv
@@ -406,6 +448,13 @@ class Replica:
             work = {"flops": work["flops"], "bytes": work["bytes"] - M * K * 0.5625 + M * K * 2.0}
             return [("linear", lambda: nv.linear(self.x["X"], self.q["W"], x_global_scale=self.x_scale,
                                                  out=self.out["C"], workspace=self.ws["lin"]), work, "gemm")]
+        if k in ("decode_lora", "prefill_lora"):
+            out = []
+            sufs = [("_up", cfg["N_up"], cfg["K_up"]), ("_down", cfg["N_down"], cfg["K_down"])] \
+                if k == "prefill_lora" else [("", cfg["N"], cfg["K"])]
+            for suf, n, kk in sufs:
+                out.append(("linear_lora" + suf, self._lora(suf), lora_work(cfg["M"], n, kk, cfg["R"]), "gemm"))
+            return out
         if k == "mse":
             return [("quantize_mse_W", lambda: nv.nvfp4_quantize(self.x["W"], "mse", out=self.q["W"],
                                                                  workspace=self.ws["W"]), qwork("W"), "quantize")]
@@ -429,7 +478,7 @@ def step_units(cfg, groups):
     """(total work of one step, unit, scale): GEMM FLOPs in TFLOP/s where the step has a
     compute-bound GEMM, otherwise algorithmic bytes in GB/s."""
     k = cfg["kind"]
-    if k in ("decode", "mse"):
+    if k in ("decode", "mse", "decode_lora"):
         return sum(w["bytes"] for _, _, w, _ in groups), "GB/s", 1e9
     return sum(w.get("flops", 0.0) for _, _, w, fam in groups if fam == "gemm"), "TFLOP/s", 1e12
 
@@ -563,10 +612,14 @@ def run_ours(args, rank, world, local, host):
     dom = max(names, key=lambda n: per_group[n])
     roof = group_rate(works[dom], per_group[dom], peaks, long_region)
     if families[dom] == "gemm":
-        n_of = {"gemm_1": "N1", "gemm_2": "N2", "gemm_up": "N_up", "gemm_down": "N_down", "gemm": "N", "linear": "N"}
+        n_of = {"gemm_1": "N1", "gemm_2": "N2", "gemm_up": "N_up", "gemm_down": "N_down", "gemm": "N", "linear": "N",
+                "linear_lora": "N", "linear_lora_up": "N_up", "linear_lora_down": "N_down"}
         kname = gemm_kernel_name(cfg["M"], cfg[n_of[dom]])
         if dom == "linear":
             kname = "gemm_decode_kernel<true> (activation quantized in the GEMM; tcgen05 mxf4nvf4, stream-K)"
+        if dom.startswith("linear_lora"):
+            kname = ("lora_down_kernel + " + ("gemm_decode_kernel<true, true>" if cfg["M"] <= 32 else
+                     "quantize_kernel + gemm_pair_kernel<true>") + " (low-rank MMAs in the FP4 accumulator)")
     else:
         kname = "amax_kernel + quantize_kernel" if dom.startswith("quantize") else "dequantize_kernel"
     roof.update({"traffic": profiled_traffic(families[dom], f"{dom}_{args.workload}"),
@@ -709,6 +762,20 @@ class OracleStep:
         t = time.perf_counter() - t0
         self.parts.append((name, n, M * N, t * (M * N) / n))
 
+    def lora(self, name, suf, M, share):
+        """The low-rank term on a row sample (t for the rows, then t B^T for all columns)."""
+        np, oracle = self.np, self.oracle
+        x, A, B = self.bits["X" + suf], self.bits["A" + suf], self.bits["B" + suf]
+        t0 = time.perf_counter()
+        oracle.lora_f64(np.ascontiguousarray(x[:1]), A, B)
+        per_row = time.perf_counter() - t0
+        n = int(min(M, max(self.threads, self.budget * share * self.threads / max(per_row, 1e-9))))
+        t0 = time.perf_counter()
+        self._pool_map(lambda ab: oracle.lora_f64(np.ascontiguousarray(x[ab[0]:ab[1]]), A, B),
+                       _split_rows(n, self.threads))
+        t = time.perf_counter() - t0
+        self.parts.append((name, n, M, t * M / n))
+
     def dequantize(self, name, q, rows_full):
         np, oracle = self.np, self.oracle
         codes, scales, sg = q
@@ -742,6 +809,14 @@ class OracleStep:
             wq = self.quantize("W", o.SCALE_ABSMAX, 0.2)
             self.parts = [p for p in self.parts if p[0] != "quantize W"]
             self.gemm("gemm", x, wq, cfg["M"], cfg["N"], 0.7)
+        elif k in ("decode_lora", "prefill_lora"):
+            sufs = [("_up", "N_up"), ("_down", "N_down")] if k == "prefill_lora" else [("", "N")]
+            for suf, nkey in sufs:
+                xq = self.quantize("X" + suf, o.SCALE_ABSMAX, 0.1 / len(sufs))
+                wq = self.quantize("W" + suf, o.SCALE_ABSMAX, 0.1 / len(sufs))
+                self.parts = [p for p in self.parts if p[0] != "quantize W" + suf]
+                self.gemm("gemm" + suf, xq, wq, cfg["M"], cfg[nkey], 0.5 / len(sufs))
+                self.lora("lora" + suf, suf, cfg["M"], 0.3 / len(sufs))
         elif k == "mse":
             self.quantize("W", o.SCALE_MSE, 1.0)
         elif k == "pr1":
@@ -751,7 +826,7 @@ class OracleStep:
         return sum(p[3] for p in self.parts)
 
     def describe(self):
-        s = "; ".join(f"{n}: {u} of {f} {'rows' if n.startswith(('quantize', 'dequantize')) else 'outputs'}"
+        s = "; ".join(f"{n}: {u} of {f} {'rows' if n.startswith(('quantize', 'dequantize', 'lora')) else 'outputs'}"
                       for n, u, f, _ in self.parts)
         return f"oracle on {self.threads} host thread(s): {s}; each part extrapolated to the full step"
 
@@ -791,6 +866,11 @@ def _static_groups(cfg):
         M, N, K = cfg["M"], cfg["N"], cfg["K"]
         w = gemm_work(M, N, K)
         return [("linear", None, {"flops": w["flops"], "bytes": w["bytes"] - M * K * 0.5625 + M * K * 2.0}, "gemm")]
+    if k == "decode_lora":
+        return [("linear_lora", None, lora_work(cfg["M"], cfg["N"], cfg["K"], cfg["R"]), "gemm")]
+    if k == "prefill_lora":
+        return [("linear_lora_up", None, lora_work(cfg["M"], cfg["N_up"], cfg["K_up"], cfg["R"]), "gemm"),
+                ("linear_lora_down", None, lora_work(cfg["M"], cfg["N_down"], cfg["K_down"], cfg["R"]), "gemm")]
     if k == "mse":
         return [("quantize_mse_W", None, q(cfg["rows"], cfg["cols"]), "quantize")]
     if k == "pr1":

@@ -185,8 +185,74 @@ nvfp4_status nvfp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, con
                           int64_t N, void *c, int64_t ldc, void *workspace, size_t workspace_bytes,
                           void *stream);
 
+/* Workspace nvfp4_linear_lora needs (device memory, any content on entry). */
+size_t nvfp4_linear_lora_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t R);
+
+/* The W4A4 linear layer with a low-rank (LoRA) branch, y = Q(x) W^T + (x A^T) B^T --
+ * the page "NVFP4 en difusión: la misma cuantización, un motor completamente
+ * distinto", section 3 ("¿Cómo fine-tuneás algo que ya está en 4 bits?"): a LoRA
+ * cannot be merged into NVFP4 weights, so the kernel computes y = W_4bit x + B (A x),
+ * the low-rank term in 16 bits, added to the quantized matmul before the result
+ * is returned.  Here t = x A^T (M x R) is accumulated in FP32 on the tensor cores
+ * and rounded to BF16 (the 16-bit intermediate); t B^T is added to the W4A4 GEMM's
+ * FP32 accumulator by tensor-core MMAs, and the sum is rounded to BF16 once.
+ *   x, M, K, ld_x, x_global_scale, w_codes, w_scales, w_global_scale, N, c, ldc:
+ *                as nvfp4_linear (the activation is quantized on the call, absmax).
+ *   lora_a       device BF16, R x K, row-major (row stride K).
+ *   lora_b       device BF16, N x R, row-major (row stride R).
+ *   R            the rank: 16, 32, 48 or 64.
+ *   t_out        device BF16 M x R (row stride R) or NULL: receives t.
+ * The order of t's FP32 accumulation is the tensor cores' (t can differ by one BF16
+ * ulp from a differently ordered sum).  The GEMM consumes t / (s_gA s_gB) as two
+ * BF16 parts (about 2^-16 relative), so alpha = s_gA s_gB must be a normal float.
+ * Errors: INVALID_ARG, SHAPE (K % 32, R), ALIGNMENT, WORKSPACE, UNSUPPORTED_DEVICE,
+ * CUDA; device-side timeouts as for nvfp4_linear. */
+nvfp4_status nvfp4_linear_lora(const void *x, int64_t M, int64_t K, int64_t ld_x, const float *x_global_scale,
+                               const uint8_t *w_codes, const uint8_t *w_scales, const float *w_global_scale,
+                               int64_t N, const void *lora_a, const void *lora_b, int64_t R, void *c, int64_t ldc,
+                               void *t_out, void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------------
+ * MXFP4 -- the microscaled 4-bit format that "Cuantización en Producción: AWQ, GPTQ,
+ * GGUF K-quants, FP8, MXFP4/NVFP4" (section "MXFP4 / NVFP4: Blackwell agresivo")
+ * names next to NVFP4 without giving its block size or scale type.  These calls
+ * follow the public OCP Microscaling Formats (MX) v1.0 specification: E2M1 codes in
+ * blocks of 32 along K, one E8M0 scale (a power of two, 2^(byte - 127)) per block, no
+ * per-tensor scale.  Codes are packed as for NVFP4; the SWIZZLED scale layout is
+ * NVFP4's 128 x 4 atom layout with one byte per 32-value block.
+ * --------------------------------------------------------------------------------- */
+
+/* Bytes of an MXFP4 scale buffer: rows x cols/32 (LINEAR) or padded to 128 rows and
+ * 4 block columns (SWIZZLED). */
+size_t mxfp4_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout);
+
+/* Quantize a BF16 matrix to MXFP4: per 32-value block, the scale 2^e with
+ * e = floor(log2 amax) - 2 clamped to [-127, 127] (byte e + 127; byte 0 for an
+ * all-zero block), codes E2M1(x / 2^e) rounded to nearest (ties to even),
+ * saturating at 6, the sign kept.
+ *   x      device BF16, rows x cols, row stride ld_x (ld_x % 8 == 0); cols % 32 == 0.
+ *   codes  device, nvfp4_codes_bytes(rows, cols) bytes.
+ *   scales device, mxfp4_scales_bytes(rows, cols, layout) bytes (padding zeroed).
+ * Bit-exact with the CPU definition shipped with the tests.  Errors: INVALID_ARG,
+ * SHAPE, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA. */
+nvfp4_status mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, nvfp4_sf_layout layout,
+                            uint8_t *codes, uint8_t *scales, void *stream);
+
+/* BF16 reconstruction q * 2^(s - 127) (exact in binary32, rounded to BF16). */
+nvfp4_status mxfp4_dequantize(const uint8_t *codes, const uint8_t *scales, nvfp4_sf_layout layout, int64_t rows,
+                              int64_t cols, void *out, int64_t ld_out, void *stream);
+
+/* The MXFP4 x MXFP4 GEMM, C = A B^T with the block scales applied inside the kernel
+ * (tcgen05 block-scaled MMA with 32-value UE8M0 scales), FP32 accumulation, BF16 out.
+ *   A: M x K (codes, SWIZZLED scales), B: N x K (the weight, out x in), C: M x N, ldc.
+ *   M, N >= 1; K % 32 == 0.  workspace: nvfp4_gemm_workspace_bytes(M, N, K) bytes.
+ * Errors as nvfp4_gemm. */
+nvfp4_status mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, int64_t M, const uint8_t *b_codes,
+                        const uint8_t *b_scales, int64_t N, int64_t K, void *c, int64_t ldc, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
 /* Synchronize `stream` and read the device status word at the start of a GEMM
- * (or nvfp4_linear) workspace.  Returns NVFP4_OK when no bounded wait gave up, NVFP4_ERR_TIMEOUT
+ * (or nvfp4_linear, nvfp4_linear_lora) workspace.  Returns NVFP4_OK when no bounded wait gave up, NVFP4_ERR_TIMEOUT
  * otherwise (and stores the raw word, which names the wait, in *word if non-NULL),
  * NVFP4_ERR_CUDA if the copy fails.  Clears nothing: a workspace is reset by the
  * next nvfp4_gemm that uses it. */

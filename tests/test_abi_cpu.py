@@ -17,7 +17,7 @@ HEADER = os.path.join(ROOT, "include", "nvfp4.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(nvfp4_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b((?:nvfp4|mxfp4)_\w+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -190,3 +190,43 @@ def test_noalloc_validation_before_any_cuda_call(lib):
     assert q(x=8) == 3
     assert q(ld=36) == 3
     assert q() in (4, 5)
+
+
+def test_linear_validation_before_any_cuda_call(lib):
+    P = ctypes.c_void_p
+
+    def g(M=8, N=256, K=64, ld=64, ldc=256, ptr=16, ws=16, ws_bytes=1 << 30, x_gs=None):
+        p = P(ptr) if ptr else None
+        return lib.nvfp4_linear(p, M, K, ld, P(x_gs) if x_gs else None, p, p, P(16), N, p, ldc,
+                                P(ws) if ws else None, ws_bytes, None)
+
+    assert g(K=48, ld=48) == 2          # K % 32
+    assert g(M=0) == 1
+    assert g(ld=32) == 1                # ld_x < K
+    assert g(ptr=0) == 1
+    assert g(ws=0) == 7
+    assert g(ws_bytes=511) == 7
+    assert g(ptr=8) == 3
+    assert g(x_gs=18) == 3
+    assert g() in (4, 5)
+    assert lib.nvfp4_linear_workspace_bytes(8, 14336, 4096) == 512 + lib.nvfp4_gemm_workspace_bytes(8, 14336, 4096) - 256
+    assert lib.nvfp4_linear_workspace_bytes(4096, 14336, 4096) >= 512 + 4096 * 2048 + 4096 * 256
+
+
+def test_linear_lora_validation_before_any_cuda_call(lib):
+    P = ctypes.c_void_p
+
+    def g(M=8, N=256, K=64, R=16, ptr=16, ws=16, ws_bytes=1 << 30, a=16, b=16, t=None):
+        p = P(ptr) if ptr else None
+        return lib.nvfp4_linear_lora(p, M, K, K, None, p, p, P(16), N, P(a) if a else None, P(b) if b else None, R,
+                                     p, N, P(t) if t else None, P(ws) if ws else None, ws_bytes, None)
+
+    assert g(R=8) == 2                  # rank not a multiple of 16
+    assert g(R=80) == 2                 # rank above 64
+    assert g(R=0) == 1
+    assert g(a=0) == 1 and g(b=0) == 1
+    assert g(ws_bytes=100) == 7
+    assert g(b=24) == 3 and g(t=40) == 3
+    assert g() in (4, 5) and g(R=64, M=4096) in (4, 5)
+    small = lib.nvfp4_linear_lora_workspace_bytes(8, 14336, 4096, 64)
+    assert small > lib.nvfp4_linear_workspace_bytes(8, 14336, 4096)

@@ -53,6 +53,12 @@ SIGNATURES = {
     "nvfp4_gemm": ([_P, _P, _P, _I64, _P, _P, _P, _I64, _I64, _P, _I64, _P, _SZ, _P], _I),
     "nvfp4_linear_workspace_bytes": ([_I64, _I64, _I64], _SZ),
     "nvfp4_linear": ([_P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, _P, _I64, _P, _SZ, _P], _I),
+    "nvfp4_linear_lora_workspace_bytes": ([_I64, _I64, _I64, _I64], _SZ),
+    "nvfp4_linear_lora": ([_P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _I64, _P, _I64, _P, _P, _SZ, _P], _I),
+    "mxfp4_scales_bytes": ([_I64, _I64, _I], _SZ),
+    "mxfp4_quantize": ([_P, _I64, _I64, _I64, _I, _P, _P, _P], _I),
+    "mxfp4_dequantize": ([_P, _P, _I, _I64, _I64, _P, _I64, _P], _I),
+    "mxfp4_gemm": ([_P, _P, _I64, _P, _P, _I64, _I64, _P, _I64, _P, _SZ, _P], _I),
     "nvfp4_read_device_error": ([_P, _P, ctypes.POINTER(ctypes.c_uint32)], _I),
     "nvfp4_last_launch_count": ([], _I),
     "nvfp4_quantize_noalloc": ([_P, _I64, _I64, _I64, _I, _I, _P, _P, _P, _P, _P, _P], _I),
@@ -250,4 +256,87 @@ def linear(x: torch.Tensor, w: NVFP4Tensor, x_global_scale: Optional[torch.Tenso
                           _ptr(w.global_scale), N, _ptr(out), out.stride(0), _ptr(workspace), workspace.numel(),
                           _stream(stream))
     _check(st, "nvfp4_linear")
+    return out
+
+
+def linear_lora(x: torch.Tensor, w: NVFP4Tensor, lora_a: torch.Tensor, lora_b: torch.Tensor,
+                x_global_scale: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                t_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """W4A4 linear layer with a low-rank branch, y = Q(x) w^T + (x A^T) B^T in BF16:
+    lora_a (R x K) and lora_b (N x R) BF16 CUDA tensors, rank R in {16, 32, 48, 64};
+    t = x A^T is rounded to BF16 (returned in t_out if given) and t B^T is added to the
+    W4A4 GEMM's FP32 accumulator before the single BF16 rounding."""
+    lib = load_library()
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D row-major bfloat16 CUDA tensor")
+    M, K = x.shape
+    N, R = w.rows, lora_a.shape[0]
+    if w.layout != SF_SWIZZLED or w.cols != K:
+        raise ValueError("w must share K with x and have swizzled scales")
+    for t, shape in ((lora_a, (R, K)), (lora_b, (N, R))):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"low-rank factors must be contiguous bfloat16 of shapes {(R, K)} and {(N, R)}")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(lib.nvfp4_linear_lora_workspace_bytes(M, N, K, R), dtype=torch.uint8,
+                                device=x.device)
+    st = lib.nvfp4_linear_lora(_ptr(x), M, K, x.stride(0), _ptr(x_global_scale), _ptr(w.codes), _ptr(w.scales),
+                               _ptr(w.global_scale), N, _ptr(lora_a), _ptr(lora_b), R, _ptr(out), out.stride(0),
+                               _ptr(t_out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "nvfp4_linear_lora")
+    return out
+
+
+@dataclass
+class MXFP4Tensor:
+    """A rows x cols tensor in MXFP4: packed E2M1 codes and one E8M0 scale per 32 values."""
+    codes: torch.Tensor   # uint8 (rows, cols/2)
+    scales: torch.Tensor  # uint8, flat swizzled buffer or (rows, cols/32) linear
+    rows: int
+    cols: int
+    layout: int = SF_SWIZZLED
+
+
+def mxfp4_quantize(x: torch.Tensor, layout="swizzled", out: Optional[MXFP4Tensor] = None, stream=None) -> MXFP4Tensor:
+    """Quantize a 2-D BF16 CUDA tensor (cols % 32 == 0) to MXFP4."""
+    lib = load_library()
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D row-major bfloat16 CUDA tensor")
+    rows, cols = x.shape
+    lay = _LAYOUTS[layout]
+    if out is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+        scales = torch.empty(lib.mxfp4_scales_bytes(rows, cols, lay), dtype=torch.uint8, device=x.device)
+        if lay == SF_LINEAR:
+            scales = scales.view(rows, cols // 32)
+        out = MXFP4Tensor(codes, scales, rows, cols, lay)
+    _check(lib.mxfp4_quantize(_ptr(x), rows, cols, x.stride(0), lay, _ptr(out.codes), _ptr(out.scales),
+                              _stream(stream)), "mxfp4_quantize")
+    return out
+
+
+def mxfp4_dequantize(q: MXFP4Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    lib = load_library()
+    if out is None:
+        out = torch.empty((q.rows, q.cols), dtype=torch.bfloat16, device=q.codes.device)
+    _check(lib.mxfp4_dequantize(_ptr(q.codes), _ptr(q.scales), q.layout, q.rows, q.cols, _ptr(out), out.stride(0),
+                                _stream(stream)), "mxfp4_dequantize")
+    return out
+
+
+def mxfp4_gemm(a: MXFP4Tensor, b: MXFP4Tensor, out: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """C = A B^T in BF16 for MXFP4 operands (A M x K, B N x K, swizzled scales)."""
+    lib = load_library()
+    if a.cols != b.cols or a.layout != SF_SWIZZLED or b.layout != SF_SWIZZLED:
+        raise ValueError("A and B must share K and have swizzled scales")
+    M, N, K = a.rows, b.rows, a.cols
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.codes.device)
+    if workspace is None:
+        workspace = torch.empty(lib.nvfp4_gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device=a.codes.device)
+    _check(lib.mxfp4_gemm(_ptr(a.codes), _ptr(a.scales), M, _ptr(b.codes), _ptr(b.scales), N, K, _ptr(out),
+                          out.stride(0), _ptr(workspace), workspace.numel(), _stream(stream)), "mxfp4_gemm")
     return out

@@ -7,7 +7,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["api.cu", "quantize.cu", "gemm_sm100.cu", "quantize_noalloc.cu"]
+SOURCES = ["api.cu", "quantize.cu", "gemm_sm100.cu", "lora.cu", "quantize_noalloc.cu"]
 LIB = os.path.join(HERE, "libnvfp4_b200.so")
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared", "-Xptxas", "-v"]

@@ -261,6 +261,168 @@ nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, int64_t ld_x, con
   return st;
 }
 
+// Workspace of nvfp4_linear_lora: the 512-byte header of nvfp4_linear, the
+// down-projection's counters, the small-M kernel's counters (one zeroed range), then
+// the down-projection's partial tiles, t / alpha hi and lo, and the GEMM's scratch
+// (small M) or the activation's codes and scales (large M).
+struct LoraLayout {
+  size_t lora_counters, gemm_scratch, lora_partial, thi, tlo, x_codes, x_scales, zero, total;
+};
+
+LoraLayout lora_layout(int64_t M, int64_t N, int64_t K, int64_t R) {
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  LoraLayout l{};
+  size_t off = kLinearHeader;
+  l.lora_counters = off;
+  off += nvfp4::lora_counter_bytes(M);
+  l.gemm_scratch = off;
+  if (M <= 32) off += nvfp4::gemm_scratch_bytes(M, N, K);
+  l.zero = M <= 32 ? l.gemm_scratch + (nvfp4::gemm_zero_bytes(M, N, K) - 256) : l.gemm_scratch;
+  off = up(off);
+  l.lora_partial = off;
+  off = up(off + nvfp4::lora_partial_bytes(M, K, R));
+  l.thi = off;
+  off = up(off + static_cast<size_t>(M * R * 2));
+  l.tlo = off;
+  off = up(off + static_cast<size_t>(M * R * 2));
+  if (M > 32) {
+    l.x_codes = off;
+    off += linear_codes_bytes(M, K);
+    l.x_scales = off;
+    off += nvfp4_scales_bytes(M, K, NVFP4_SF_SWIZZLED);
+  }
+  l.total = off;
+  return l;
+}
+
+size_t nvfp4_linear_lora_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t R) {
+  if (M < 1 || N < 1 || K < 1 || R < 1) return kLinearHeader;
+  return lora_layout(M, N, K, R).total;
+}
+
+nvfp4_status nvfp4_linear_lora(const void* x, int64_t M, int64_t K, int64_t ld_x, const float* x_global_scale,
+                               const uint8_t* w_codes, const uint8_t* w_scales, const float* w_global_scale,
+                               int64_t N, const void* lora_a, const void* lora_b, int64_t R, void* c, int64_t ldc,
+                               void* t_out, void* workspace, size_t workspace_bytes, void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (M < 1 || N < 1 || K < 1 || ld_x < K || ldc < N || R < 1) return NVFP4_ERR_INVALID_ARG;
+  if (K % 32 != 0 || R % 16 != 0 || R > 64 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
+    return NVFP4_ERR_SHAPE;
+  if (!x || !w_codes || !w_scales || !w_global_scale || !c || !lora_a || !lora_b) return NVFP4_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < nvfp4_linear_lora_workspace_bytes(M, N, K, R)) return NVFP4_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(c) || !aligned16(workspace) ||
+      !aligned16(lora_a) || !aligned16(lora_b) || (t_out && !aligned16(t_out)) || ld_x % 8 != 0 ||
+      ldc % 8 != 0 || (reinterpret_cast<uintptr_t>(w_global_scale) & 3u) ||
+      (x_global_scale && (reinterpret_cast<uintptr_t>(x_global_scale) & 3u)))
+    return NVFP4_ERR_ALIGNMENT;
+  nvfp4_status st = check_device_cached();
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const LoraLayout l = lora_layout(M, N, K, R);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  uint32_t* amax_word = reinterpret_cast<uint32_t*>(ws + 256);
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  uint16_t* thi = reinterpret_cast<uint16_t*>(ws + l.thi);
+  uint16_t* tlo = reinterpret_cast<uint16_t*>(ws + l.tlo);
+  if (cudaMemsetAsync(ws, 0, l.zero, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (x_global_scale == nullptr) {
+    st = from_cuda(nvfp4::launch_amax(xb, M, K, ld_x, amax_word, s));
+    if (st != NVFP4_OK) return st;
+    ++nvfp4::g_last_launches;
+  }
+  st = from_cuda(nvfp4::launch_lora_down(xb, M, K, ld_x, x_global_scale, x_global_scale ? nullptr : amax_word,
+                                         w_global_scale, static_cast<const uint16_t*>(lora_a), R,
+                                         static_cast<uint16_t*>(t_out), thi, tlo,
+                                         reinterpret_cast<uint32_t*>(ws + l.lora_counters),
+                                         reinterpret_cast<float*>(ws + l.lora_partial), status, s));
+  if (st != NVFP4_OK) return st;
+  ++nvfp4::g_last_launches;
+  const uint16_t* lb = static_cast<const uint16_t*>(lora_b);
+  if (M <= 32) {
+    st = from_cuda(nvfp4::launch_decode_quantize_x_lora(
+        xb, M, K, ld_x, x_global_scale, x_global_scale ? nullptr : amax_word, w_codes, w_scales, w_global_scale, N,
+        lb, thi, tlo, R, static_cast<uint16_t*>(c), ldc, status, ws + l.gemm_scratch, s));
+    if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+    return st;
+  }
+  float* a_gs = x_global_scale ? nullptr : reinterpret_cast<float*>(ws + 260);
+  st = from_cuda(nvfp4::launch_quantize(xb, M, K, ld_x, NVFP4_SCALE_ABSMAX, true, x_global_scale, amax_word,
+                                        ws + l.x_codes, ws + l.x_scales, a_gs, nullptr, s));
+  if (st != NVFP4_OK) return st;
+  ++nvfp4::g_last_launches;
+  st = from_cuda(nvfp4::launch_gemm_lora(ws + l.x_codes, ws + l.x_scales, x_global_scale ? x_global_scale : a_gs, M,
+                                         w_codes, w_scales, w_global_scale, N, K, static_cast<uint16_t*>(c), ldc,
+                                         status, lb, thi, tlo, R, s));
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
+}
+
+size_t mxfp4_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout) {
+  if (rows < 0 || cols < 0) return 0;
+  const int64_t nblk = cols / 32;
+  if (layout == NVFP4_SF_LINEAR) return static_cast<size_t>(rows * nblk);
+  return static_cast<size_t>((rows + 127) / 128 * 128 * ((nblk + 3) / 4 * 4));
+}
+
+nvfp4_status mxfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld_x, nvfp4_sf_layout layout,
+                            uint8_t* codes, uint8_t* scales, void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (rows < 0 || cols < 0 || ld_x < cols) return NVFP4_ERR_INVALID_ARG;
+  if (layout != NVFP4_SF_SWIZZLED && layout != NVFP4_SF_LINEAR) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 32 != 0) return NVFP4_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (!x || !codes || !scales) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || ld_x % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+  nvfp4_status st = check_device_cached();
+  if (st != NVFP4_OK) return st;
+  st = from_cuda(nvfp4::launch_quantize_mx(static_cast<const uint16_t*>(x), rows, cols, ld_x,
+                                           layout == NVFP4_SF_SWIZZLED, codes, scales,
+                                           static_cast<cudaStream_t>(stream)));
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
+}
+
+nvfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, nvfp4_sf_layout layout, int64_t rows,
+                              int64_t cols, void* out, int64_t ld_out, void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (rows < 0 || cols < 0 || ld_out < cols) return NVFP4_ERR_INVALID_ARG;
+  if (layout != NVFP4_SF_SWIZZLED && layout != NVFP4_SF_LINEAR) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 32 != 0) return NVFP4_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (!codes || !scales || !out) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(out) || ld_out % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+  nvfp4_status st = check_device_cached();
+  if (st != NVFP4_OK) return st;
+  st = from_cuda(nvfp4::launch_dequantize_mx(codes, scales, layout == NVFP4_SF_SWIZZLED, rows, cols,
+                                             static_cast<uint16_t*>(out), ld_out, static_cast<cudaStream_t>(stream)));
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
+}
+
+nvfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M, const uint8_t* b_codes,
+                        const uint8_t* b_scales, int64_t N, int64_t K, void* c, int64_t ldc, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (M < 1 || N < 1 || K < 1 || ldc < N) return NVFP4_ERR_INVALID_ARG;
+  if (K % 32 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return NVFP4_ERR_SHAPE;
+  if (!a_codes || !a_scales || !b_codes || !b_scales || !c) return NVFP4_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < nvfp4_gemm_workspace_bytes(M, N, K)) return NVFP4_ERR_WORKSPACE;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) || !aligned16(c) ||
+      !aligned16(workspace) || ldc % 8 != 0)
+    return NVFP4_ERR_ALIGNMENT;
+  nvfp4_status st = check_device_cached();
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the status word (and the small-M kernel's counters) cleared before the kernel
+  if (cudaMemsetAsync(workspace, 0, M <= 32 ? nvfp4::gemm_zero_bytes(M, N, K) : 256, s) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  st = from_cuda(nvfp4::launch_gemm_mx(a_codes, a_scales, M, b_codes, b_scales, N, K, static_cast<uint16_t*>(c), ldc,
+                                       static_cast<uint32_t*>(workspace), s));
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
+}
+
 nvfp4_status nvfp4_read_device_error(const void* workspace, void* stream, uint32_t* word) {
   if (!workspace) return NVFP4_ERR_INVALID_ARG;
   uint32_t w = 0;

@@ -331,11 +331,12 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 // bytes before it arrives, so the MMA issuer waits on one barrier per K-tile: every
 // wait in the issuing thread lets the tensor pipe's queue run dry (with four MMAs
 // per wait the pipe already runs at about 85 % of its rate).  The peer's set
-// gathers its four warps on a local barrier and one of them arrives with a
-// cluster-scope release, which orders the set's TMEM stores before the leader's MMA
-// reads them (one remote release per K-tile: four of them cost ~10 % of the GEMM).
+// gathers its four warps on a local barrier -- every warp waits for the phase, so
+// that no warp's next arrival can complete it early -- and one of them arrives with
+// a cluster-scope release, which orders the set's TMEM stores before the leader's
+// MMA reads them (one remote release per K-tile: four of them cost ~10 % of the GEMM).
 // Scale factors have their own producer and shared-memory slots, refilled as soon
-// as a set has read them, so they land several K-tiles ahead of their MMAs.  A stage's region is free again when its shared-memory
+// as a set has moved them to TMEM, so they land several K-tiles ahead of their MMAs.  A stage's region is free again when its shared-memory
 // slot is: the producer reloads stage s only after the MMAs that read it
 // completed, so no separate release barrier is needed.  Each K-tile's MMAs end with
 // one commit that arrives on both CTAs' `empty` barriers.
@@ -345,6 +346,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 // reads), and write BF16 through 128-byte-swizzled shared-memory boxes with TMA
 // stores.
 
+template <bool LR = false>
 struct PairCfg {
   static constexpr int BM = 128;                      // rows of A per CTA (256 per pair)
   static constexpr int BN = 256;                      // columns of the pair's tile
@@ -355,12 +357,16 @@ struct PairCfg {
   static constexpr int SFA_BYTES = 4 * SF_ATOM;       // own 128 rows, 4 K-steps
   static constexpr int SFB_BYTES = 2 * 4 * SF_ATOM;   // all 256 rows, 4 K-steps
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = 5;
+  // LR (low-rank branch): four stages, C written with direct stores (no staging boxes),
+  // and the tile's low-rank operands -- t / alpha hi and lo (this CTA's 128 rows) and
+  // B's rows (this CTA's 128 columns), 128-byte K-major rows (rank up to 64)
+  static constexpr int STAGES = LR ? 4 : 5;
   static constexpr int EPI_WARPS = 8;
   static constexpr int C_BOX_BYTES = 32 * 128;        // 32 rows x 64 BF16 columns
-  static constexpr int C_BYTES = EPI_WARPS * C_BOX_BYTES;
+  static constexpr int C_BYTES = LR ? 0 : EPI_WARPS * C_BOX_BYTES;
+  static constexpr int LORA_BYTES = LR ? 3 * 128 * 128 : 0;
   static constexpr int BAR_BYTES = 512;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + C_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + C_BYTES + LORA_BYTES + BAR_BYTES;
   static constexpr int PRODUCER_WARP = EPI_WARPS;     // 8
   static constexpr int MMA_WARP = EPI_WARPS + 1;      // 9
   static constexpr int SF_WARP0 = EPI_WARPS + 2;      // 10..
@@ -376,19 +382,25 @@ struct PairCfg {
   static_assert(BN + SF_REGIONS * SF_COLS <= TMEM_COLS, "TMEM budget");
 };
 
-__global__ void __launch_bounds__(PairCfg::THREADS, 1)
+template <bool LR, bool MX>
+__global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                     const __grid_constant__ CUtensorMap tmap_c, const float* __restrict__ a_gs,
+                     const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_lb,
+                     const __grid_constant__ CUtensorMap tmap_thi, const __grid_constant__ CUtensorMap tmap_tlo,
+                     int rank_lr, uint16_t* __restrict__ C, int64_t ldc, const float* __restrict__ a_gs,
                      const float* __restrict__ b_gs, int M, int N, int K, uint32_t* __restrict__ status) {
-  using Cfg = PairCfg;
+  using Cfg = PairCfg<LR>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int R = Cfg::SF_REGIONS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * Cfg::A_BYTES;
-  uint8_t* sSFA = sB + STAGES * Cfg::B_BYTES;
+  uint8_t* sLB = sB + STAGES * Cfg::B_BYTES;            // LR: B's rows, then t / alpha hi and lo
+  uint8_t* sTH = sLB + Cfg::LORA_BYTES / 3;
+  uint8_t* sTL = sTH + Cfg::LORA_BYTES / 3;
+  uint8_t* sSFA = sLB + Cfg::LORA_BYTES;
   uint8_t* sSFB = sSFA + STAGES * Cfg::SFA_BYTES;
   uint8_t* sC = sSFB + STAGES * Cfg::SFB_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sC + Cfg::C_BYTES);
@@ -400,7 +412,9 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
   uint64_t* acc_full = set_done + Cfg::SF_SETS;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* lora_full = drain + 1;    // LR, leader: the tile's low-rank operands landed (both CTAs)
+  uint64_t* lora_empty = lora_full + 1;  // LR, both CTAs: the low-rank MMAs completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lora_empty + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -425,6 +439,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * Cfg::EPI_WARPS);
     mbar_init(drain, 1);
+    mbar_init(lora_full, 1);
+    mbar_init(lora_empty, 1);
     *abort_flag = 0u;
     fence_mbarrier_init();
   }
@@ -437,7 +453,13 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     prefetch_tmap(&tmap_b);
     prefetch_tmap(&tmap_sfa);
     prefetch_tmap(&tmap_sfb);
-    prefetch_tmap(&tmap_c);
+    if (LR) {
+      prefetch_tmap(&tmap_lb);
+      prefetch_tmap(&tmap_thi);
+      prefetch_tmap(&tmap_tlo);
+    } else {
+      prefetch_tmap(&tmap_c);
+    }
   }
   tc_fence_before();
   __syncwarp();
@@ -454,11 +476,24 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       int issued_last[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
-      int kc = 0;
+      int kc = 0, it = 0;
       bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += npairs) {
+      for (int t = pair; t < num_tiles && ok; t += npairs, ++it) {
         int tm, tn;
         tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
+        if (LR) {
+          // the tile's low-rank operands, once the previous tile's low-rank MMAs are done
+          if (!mbar_wait_cluster(lora_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, status,
+                                 kErrWaitEmpty + 3)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(lora_full, 2u * Cfg::LORA_BYTES);
+          const uint32_t lbar = mapa_shared(smem_u32(lora_full), 0u);
+          tma_load_2d_pair(sLB, &tmap_lb, lbar, 0, tn * Cfg::BN + static_cast<int>(rank) * 128);
+          tma_load_2d_pair(sTH, &tmap_thi, lbar, 0, tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM);
+          tma_load_2d_pair(sTL, &tmap_tlo, lbar, 0, tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM);
+        }
         for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
           const int s = kc % STAGES;
           const uint32_t ph = static_cast<uint32_t>(kc / STAGES) & 1u;
@@ -481,12 +516,13 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             const uint32_t par = static_cast<uint32_t>(issued_last[s] / STAGES) & 1u;
             if (rank == 0) mbar_wait_drain(&full[s], par, status);
           }
+        if (LR && rank == 0 && it > 0) mbar_wait_drain(lora_full, static_cast<uint32_t>(it - 1) & 1u, status);
       }
     }
   } else if (warp == Cfg::MMA_WARP) {
     if (lane == 0 && rank == 0) {
       // ---------------- MMA issuer (leader CTA only) ----------------
-      const uint32_t idesc = idesc_mxf4nvf4(2 * Cfg::BM, Cfg::BN);
+      const uint32_t idesc = MX ? idesc_mxf4_e8m0(2 * Cfg::BM, Cfg::BN) : idesc_mxf4nvf4(2 * Cfg::BM, Cfg::BN);
       const uint32_t t_acc = tmem_base;
       const uint32_t acc_full_own = smem_u32(acc_full);
       bool ok = true;
@@ -498,6 +534,29 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           break;
         }
         tc_fence_after();
+        if (LR) {
+          // D += (t / alpha)(B rows)^T, hi then lo: 256 x 256 x 16 BF16 MMAs over the rank
+          if (!mbar_wait_cluster(lora_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, kErrWaitFull + 8)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t idesc_lr = idesc_bf16(2 * Cfg::BM, Cfg::BN);
+          const uint32_t lb = smem_u32(sLB), th = smem_u32(sTH), tl = smem_u32(sTL);
+          for (int kk = 0; kk < (rank_lr + 15) / 16; ++kk)
+            mma_bf16_pair(t_acc, sdesc_kmajor_sw128(th + 32 * kk), sdesc_kmajor_sw128(lb + 32 * kk), idesc_lr,
+                          kk != 0 ? 1u : 0u);
+          for (int kk = 0; kk < (rank_lr + 15) / 16; ++kk)
+            mma_bf16_pair(t_acc, sdesc_kmajor_sw128(tl + 32 * kk), sdesc_kmajor_sw128(lb + 32 * kk), idesc_lr, 1u);
+          tc_commit_pair_both(smem_u32(lora_empty));
+          // MMAs of different shapes on one accumulator are not ordered by issue: the
+          // 256 x 256 x 64 FP4 MMAs may start only once these K = 16 MMAs have completed
+          if (!mbar_wait_cluster(lora_empty, static_cast<uint32_t>(it) & 1u, abort_flag, status, kErrWaitFull + 9)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
         for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
           const int s = kc % STAGES;
           const int r = s;
@@ -513,9 +572,14 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
           const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
           const uint32_t t_sf = tmem_base + Cfg::TMEM_SF + r * Cfg::SF_COLS;
-          for (int j = 0; j < na; ++j)
-            mma_mxf4nvf4_pair(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j),
-                              idesc, t_sf + 4 * j, t_sf + 16 + 8 * j, (kt | j) != 0 ? 1u : 0u);
+          for (int j = 0; j < na; ++j) {
+            if constexpr (MX)
+              mma_mxf4_block32_pair(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j),
+                                    idesc, t_sf + 4 * j, t_sf + 16 + 8 * j, (LR || (kt | j) != 0) ? 1u : 0u);
+            else
+              mma_mxf4nvf4_pair(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j),
+                                idesc, t_sf + 4 * j, t_sf + 16 + 8 * j, (LR || (kt | j) != 0) ? 1u : 0u);
+          }
           tc_commit_pair_both(smem_u32(&empty[s]));
         }
         if (!ok) break;
@@ -529,7 +593,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
   } else if (warp == Cfg::SF_PRODUCER_WARP) {
     if (lane == 0) {
       // ---------------- scale-factor producer (both CTAs) ----------------
-      // Slot s is refilled as soon as the set that copied K-tile kc-5 has read it,
+      // Slot s is refilled as soon as the set that copied K-tile kc-STAGES has moved it to TMEM,
       // several K-tiles before the MMAs reach kc, so the scale copy is not on the
       // critical path of a stage's reload.
       int issued_last[STAGES];
@@ -547,9 +611,12 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&sf_full[s], Cfg::SFA_BYTES + Cfg::SFB_BYTES);
-          tma_load_3d(sSFA + s * Cfg::SFA_BYTES, &tmap_sfa, &sf_full[s], 0, kt * 4, tm * 2 + static_cast<int>(rank));
-          tma_load_3d(sSFB + s * Cfg::SFB_BYTES, &tmap_sfb, &sf_full[s], 0, kt * 4, tn * 2);
+          // a K-tile's scales: four 64-value atoms (NVFP4) or two 128-value atoms (MXFP4)
+          constexpr int kAtoms = MX ? 2 : 4;
+          mbar_arrive_expect_tx(&sf_full[s], (Cfg::SFA_BYTES + Cfg::SFB_BYTES) * kAtoms / 4);
+          tma_load_3d(sSFA + s * Cfg::SFA_BYTES, &tmap_sfa, &sf_full[s], 0, kt * kAtoms,
+                      tm * 2 + static_cast<int>(rank));
+          tma_load_3d(sSFB + s * Cfg::SFB_BYTES, &tmap_sfb, &sf_full[s], 0, kt * kAtoms, tn * 2);
           issued_last[s] = kc;
         }
       }
@@ -570,9 +637,9 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         if (kc % Cfg::SF_SETS != set) continue;
         const int s = kc % STAGES;
         const int r = s;
-        const uint32_t prev = (static_cast<uint32_t>(kc / STAGES) & 1u) ^ 1u;  // parity of K-tile kc-5's phase
+        const uint32_t prev = (static_cast<uint32_t>(kc / STAGES) & 1u) ^ 1u;  // parity of K-tile kc-STAGES's phase
         // A parity wait is only sound when the barrier is at most one phase behind, and
-        // the sets rotate: first see K-tile kc-5 through slot s (its set has read the
+        // the sets rotate: first see K-tile kc-STAGES through slot s (its set has read the
         // slot, so those scales had landed), then wait for kc's scales.
         if (kc >= STAGES &&
             !warp_wait(&sf_empty[s], prev, abort_flag, status, kErrWaitFull + 3)) {
@@ -586,25 +653,45 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         const uint8_t* fa = sSFA + s * Cfg::SFA_BYTES + lane * 16;
         const uint8_t* fb = sSFB + s * Cfg::SFB_BYTES + lane * 16;
         uint32_t va[16], vb[32];
+        if constexpr (MX) {
+          // MXFP4: an atom covers two MMAs (K = 128); MMA j reads its two block-32 scale
+          // bytes from the low half of its words (scale-factor id 0)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 a4 = *reinterpret_cast<const uint4*>(fa + j * Cfg::SF_ATOM);
-          va[4 * j] = a4.x;
-          va[4 * j + 1] = a4.y;
-          va[4 * j + 2] = a4.z;
-          va[4 * j + 3] = a4.w;
+          for (int j = 0; j < 4; ++j) {
+            const int sh = 16 * (j & 1);
+            const uint4 a4 = *reinterpret_cast<const uint4*>(fa + (j >> 1) * Cfg::SF_ATOM);
+            va[4 * j] = (a4.x >> sh) & 0xFFFFu;
+            va[4 * j + 1] = (a4.y >> sh) & 0xFFFFu;
+            va[4 * j + 2] = (a4.z >> sh) & 0xFFFFu;
+            va[4 * j + 3] = (a4.w >> sh) & 0xFFFFu;
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const uint4 b4 = *reinterpret_cast<const uint4*>(fb + (g * 4 + j) * Cfg::SF_ATOM);
-            vb[8 * j + 4 * g] = b4.x;
-            vb[8 * j + 4 * g + 1] = b4.y;
-            vb[8 * j + 4 * g + 2] = b4.z;
-            vb[8 * j + 4 * g + 3] = b4.w;
+            for (int g = 0; g < 2; ++g) {
+              const uint4 b4 = *reinterpret_cast<const uint4*>(fb + (g * 2 + (j >> 1)) * Cfg::SF_ATOM);
+              vb[8 * j + 4 * g] = (b4.x >> sh) & 0xFFFFu;
+              vb[8 * j + 4 * g + 1] = (b4.y >> sh) & 0xFFFFu;
+              vb[8 * j + 4 * g + 2] = (b4.z >> sh) & 0xFFFFu;
+              vb[8 * j + 4 * g + 3] = (b4.w >> sh) & 0xFFFFu;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 a4 = *reinterpret_cast<const uint4*>(fa + j * Cfg::SF_ATOM);
+            va[4 * j] = a4.x;
+            va[4 * j + 1] = a4.y;
+            va[4 * j + 2] = a4.z;
+            va[4 * j + 3] = a4.w;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              const uint4 b4 = *reinterpret_cast<const uint4*>(fb + (g * 4 + j) * Cfg::SF_ATOM);
+              vb[8 * j + 4 * g] = b4.x;
+              vb[8 * j + 4 * g + 1] = b4.y;
+              vb[8 * j + 4 * g + 2] = b4.z;
+              vb[8 * j + 4 * g + 3] = b4.w;
+            }
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sf_empty[s]);  // the slot may be refilled
-        // TMEM region r is free once the MMAs of K-tile kc-5 have completed
+        // TMEM region r is free once the MMAs of K-tile kc-STAGES have completed
         if (kc >= STAGES && !warp_wait_cluster(&empty[s], prev, abort_flag, status, kErrWaitFull + 4)) {
           ok = false;
           break;
@@ -614,6 +701,13 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
         tmem_st_32x32b_x16(t_sf, va);
         tmem_st_32x32b_x32(t_sf + 16, vb);
         tmem_st_wait();
+        // Only now may the slot be refilled: the TMEM stores consumed every value this
+        // warp loaded from it.  Releasing the slot right after issuing the loads let a
+        // load still queued behind other memory traffic (the epilogue's stores) return
+        // the next K-tile's scales, written by the refill.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_empty[s]);
         if (rank == 0 && !warp_wait_cluster(&full[s], static_cast<uint32_t>(kc / STAGES) & 1u, abort_flag, status,
                                             kErrWaitFull)) {
           ok = false;
@@ -625,14 +719,16 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           if (lane == 0) mbar_arrive(&sf_ready[r]);
         } else {
           if (lane == 0) mbar_arrive(&set_done[set]);
-          if (quarter == static_cast<uint32_t>(set & 3)) {  // one warp of the set
-            const uint32_t hand = static_cast<uint32_t>(handled & 1);
-            if (!warp_wait(&set_done[set], hand, abort_flag, status, kErrWaitFull + 5)) {
-              ok = false;
-              break;
-            }
-            if (lane == 0) mbar_arrive_cluster(sf_ready_leader0 + r * 8u);
+          // All four warps wait for the phase: a warp that went on to its next K-tile
+          // without waiting could arrive inside this phase and complete it while a
+          // slower warp of the set has not yet written its lanes.
+          if (!warp_wait(&set_done[set], static_cast<uint32_t>(handled & 1), abort_flag, status,
+                         kErrWaitFull + 5)) {
+            ok = false;
+            break;
           }
+          if (quarter == static_cast<uint32_t>(set & 3) && lane == 0)  // one warp of the set
+            mbar_arrive_cluster(sf_ready_leader0 + r * 8u);
         }
         ++handled;
       }
@@ -641,7 +737,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     // ---------------- epilogue (warps 0-7, both CTAs) ----------------
     constexpr int HALF = Cfg::BN / 2;
     const int quarter = warp & 3, half = warp >> 2;
-    const float alpha = __fmul_rn(*a_gs, *b_gs);
+    const float alpha = MX ? 1.0f : __fmul_rn(*a_gs, *b_gs);  // MXFP4 has no per-tensor scales
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * HALF;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0u);
     uint8_t* box = sC + warp * Cfg::C_BOX_BYTES;
@@ -673,6 +769,21 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       }
       const int row0 = tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM + quarter * 32;
       const int col0 = tn * Cfg::BN + half * HALF;
+      if constexpr (LR) {
+        // row row0 + lane, columns [col0, col0 + 128): 16-byte stores from registers
+        const int row = row0 + lane;
+        if (row < M && col0 < N) {
+          uint16_t* dst = C + static_cast<int64_t>(row) * ldc + col0;
+          if (col0 + HALF <= N) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int i = 0; i < HALF / 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          } else {
+            for (int i = 0; i < HALF; ++i)
+              if (col0 + i < N) dst[i] = static_cast<uint16_t>((i & 1) ? (p[i >> 1] >> 16) : (p[i >> 1] & 0xFFFFu));
+          }
+        }
+      } else {
 #pragma unroll
       for (int chunk = 0; chunk < 2; ++chunk) {
         // the previous TMA store from this box must have read it
@@ -694,6 +805,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           bulk_commit_group();
         }
         stored = true;
+      }
       }
     }
     if (lane == 0) bulk_wait_all();
@@ -749,7 +861,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 // moves the stage's scales to TMEM.  The arithmetic is the quantizer's absmax path,
 // operation for operation.
 
-template <bool QX>
+template <bool QX, bool LR = false>
 struct DecodeCfg {
   static constexpr int BM = 128;                 // weight rows per tile
   static constexpr int BN = 32;                  // activation rows (padded)
@@ -763,7 +875,11 @@ struct DecodeCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = 8;
   static constexpr int TABLE_BYTES = QX ? static_cast<int>(sizeof(ScaleTables)) : 0;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + TABLE_BYTES + 512;
+  // LR (low-rank branch): the weight tile's rows of B (128 x R) and t / alpha as hi and
+  // lo BF16 parts (32 x R each), K-major 128-byte rows (rank up to 64)
+  static constexpr int LB_BYTES = LR ? BM * 128 : 0;
+  static constexpr int LT_BYTES = LR ? BN * 128 : 0;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + LB_BYTES + 2 * LT_BYTES + TABLE_BYTES + 512;
   static constexpr int SF_WARP0 = 6;
   static constexpr int SF_GROUPS = QX ? 2 : 1;   // groups of four scale (quantizer) warps
   static constexpr int THREADS = (SF_WARP0 + 4 * SF_GROUPS) * 32;  // 0-3 epilogue, 4 producer, 5 MMA
@@ -836,23 +952,28 @@ __device__ __forceinline__ float decode_x_scale(const float* x_gs_in, const uint
   return global_scale(x_gs_in, x_amax);
 }
 
-template <bool QX>
-__global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
+template <bool QX, bool LR, bool MX>
+__global__ void __launch_bounds__(DecodeCfg<QX, LR>::THREADS)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                       const __grid_constant__ CUtensorMap tmap_lb, const __grid_constant__ CUtensorMap tmap_thi,
+                       const __grid_constant__ CUtensorMap tmap_tlo, int rank,
                        const uint8_t* __restrict__ sf_w, const uint8_t* __restrict__ sf_x,
                        const float* __restrict__ a_gs, const float* __restrict__ b_gs,
                        const uint16_t* __restrict__ xq, int64_t ld_x, const float* __restrict__ x_gs_in,
                        const uint32_t* __restrict__ x_amax, uint16_t* __restrict__ C, int M, int N, int K,
                        int64_t ldc, int max_seg, float* __restrict__ partial, uint32_t* __restrict__ counters,
                        uint32_t* __restrict__ status) {
-  using Cfg = DecodeCfg<QX>;
+  using Cfg = DecodeCfg<QX, LR>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // every 128-byte-swizzled tile (A, B) starts on a 1024-byte boundary
+  // every 128-byte-swizzled tile (A, B, the low-rank operands) starts on a 1024-byte boundary
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * Cfg::A_BYTES;
-  uint8_t* sSFA = sB + STAGES * Cfg::B_BYTES;
+  uint8_t* sLB = sB + STAGES * Cfg::B_BYTES;
+  uint8_t* sTH = sLB + Cfg::LB_BYTES;
+  uint8_t* sTL = sTH + Cfg::LT_BYTES;
+  uint8_t* sSFA = sTL + Cfg::LT_BYTES;
   uint8_t* sSFB = sSFA + STAGES * Cfg::SFA_BYTES;
   ScaleTables* tab = reinterpret_cast<ScaleTables*>(sSFB + STAGES * Cfg::SFB_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * Cfg::SFB_BYTES + Cfg::TABLE_BYTES);
@@ -862,7 +983,9 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
   uint64_t* acc_full = qdone + STAGES;     // [2]
   uint64_t* acc_empty = acc_full + 2;      // [2]
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* lora_full = drain + 1;         // LR: the low-rank operands of a tile landed
+  uint64_t* lora_empty = lora_full + 1;    // LR: their MMAs completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lora_empty + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* decision = tmem_slot + 2;
 
@@ -882,6 +1005,8 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
       mbar_init(&sf_ready[s], 4);  // lane 0 of each warp of the scale group
       mbar_init(&qdone[s], 4);
     }
+    mbar_init(lora_full, 1);
+    mbar_init(lora_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4);  // lane 0 of each epilogue warp
@@ -906,6 +1031,11 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
   if (warp == 4 && lane == 0) {
     prefetch_tmap(&tmap_w);
     if (!QX) prefetch_tmap(&tmap_x);
+    if (LR) {
+      prefetch_tmap(&tmap_lb);
+      prefetch_tmap(&tmap_thi);
+      prefetch_tmap(&tmap_tlo);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -923,7 +1053,22 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
       for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
       int64_t i = 0, s0, s1;
       bool ok = true;
+      int lora_uses = 0;
       for (int sg = 0; ok && decode_segment(sg, u0, u1, KT, s0, s1); ++sg) {
+        if (LR && s0 % KT == 0) {
+          // the segment that starts the tile's K loop also adds the low-rank term: B's rows
+          // of this tile and t / alpha (hi, lo), values past the rank and rows past M as zeros
+          if (!mbar_wait(lora_empty, (static_cast<uint32_t>(lora_uses) & 1u) ^ 1u, abort_flag, status,
+                         kErrWaitEmpty + 3)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(lora_full, Cfg::LB_BYTES + 2 * Cfg::LT_BYTES);
+          tma_load_2d(sLB, &tmap_lb, lora_full, 0, static_cast<int>(s0 / KT) * Cfg::BM);
+          tma_load_2d(sTH, &tmap_thi, lora_full, 0, 0);
+          tma_load_2d(sTL, &tmap_tlo, lora_full, 0, 0);
+          ++lora_uses;
+        }
         for (int64_t u = s0; u < s1; ++u, ++i) {
           const int s = static_cast<int>(i % STAGES);
           if (!mbar_wait(&empty[s], (static_cast<uint32_t>(i / STAGES) & 1u) ^ 1u, abort_flag, status,
@@ -932,8 +1077,11 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
             break;
           }
           const int tile = static_cast<int>(u / KT), kt = static_cast<int>(u - tile * KT);
-          const int ka0 = kt * 4;
-          const int na = min(4, k_atoms - ka0);
+          // scale atoms of the K-tile: four of 64 values (NVFP4) or two of 128 values (MXFP4)
+          constexpr int kAtoms = MX ? 2 : 4;
+          const int sf_atoms = MX ? (K + 127) / 128 : k_atoms;
+          const int ka0 = kt * kAtoms;
+          const int na = min(kAtoms, sf_atoms - ka0);
           const uint32_t sf_bytes = static_cast<uint32_t>(na) * Cfg::SF_ATOM;
           if constexpr (QX) {
             mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + sf_bytes);
@@ -941,7 +1089,7 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
             mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + 2 * sf_bytes);
           }
           tma_load_2d(sA + s * Cfg::A_BYTES, &tmap_w, &full[s], kt * Cfg::KTILE_BYTES, tile * Cfg::BM);
-          bulk_load(sSFA + s * Cfg::SFA_BYTES, sf_w + (static_cast<size_t>(tile) * k_atoms + ka0) * Cfg::SF_ATOM,
+          bulk_load(sSFA + s * Cfg::SFA_BYTES, sf_w + (static_cast<size_t>(tile) * sf_atoms + ka0) * Cfg::SF_ATOM,
                     sf_bytes, &full[s]);
           if constexpr (!QX) {
             tma_load_2d(sB + s * Cfg::B_BYTES, &tmap_x, &full[s], kt * Cfg::KTILE_BYTES, 0);
@@ -954,14 +1102,16 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
         for (int s = 0; s < STAGES; ++s)
           if (issued_last[s] >= 0)
             mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_last[s] / STAGES) & 1u, status);
+        if (LR && lora_uses > 0) mbar_wait_drain(lora_full, static_cast<uint32_t>(lora_uses - 1) & 1u, status);
       }
     }
   } else if (warp == 5) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      const uint32_t idesc = idesc_mxf4nvf4(Cfg::BM, Cfg::BN);
+      const uint32_t idesc = MX ? idesc_mxf4_e8m0(Cfg::BM, Cfg::BN) : idesc_mxf4nvf4(Cfg::BM, Cfg::BN);
       bool ok = true;
       int64_t i = 0, s0, s1;
+      int lora_uses = 0;
       for (int q = 0; ok && decode_segment(q, u0, u1, KT, s0, s1); ++q) {
         const int buf = q & 1;
         if (q >= 2) {
@@ -973,6 +1123,32 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
           tc_fence_after();
         }
         const uint32_t t_acc = tmem_base + Cfg::TMEM_ACC + buf * Cfg::BN;
+        bool lora_in = false;
+        if (LR && s0 % KT == 0) {
+          // D^T += B_rows (t/alpha)^T in two parts, hi then lo: 128 x 32 x 16 BF16 MMAs over the rank
+          if (!mbar_wait(lora_full, static_cast<uint32_t>(lora_uses) & 1u, abort_flag, status, kErrWaitFull + 8)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t idesc_lr = idesc_bf16(Cfg::BM, Cfg::BN);
+          const uint32_t lb = smem_u32(sLB), th = smem_u32(sTH), tl = smem_u32(sTL);
+          for (int kk = 0; kk < (rank + 15) / 16; ++kk)
+            mma_bf16(t_acc, sdesc_kmajor_sw128(lb + 32 * kk), sdesc_kmajor_sw128(th + 32 * kk), idesc_lr,
+                     kk != 0 ? 1u : 0u);
+          for (int kk = 0; kk < (rank + 15) / 16; ++kk)
+            mma_bf16(t_acc, sdesc_kmajor_sw128(lb + 32 * kk), sdesc_kmajor_sw128(tl + 32 * kk), idesc_lr, 1u);
+          tc_commit(lora_empty);
+          // MMAs of different shapes on one accumulator are not ordered by issue: the
+          // 128 x 32 x 64 FP4 MMAs may start only once these K = 16 MMAs have completed
+          if (!mbar_wait(lora_empty, static_cast<uint32_t>(lora_uses) & 1u, abort_flag, status, kErrWaitFull + 9)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          ++lora_uses;
+          lora_in = true;
+        }
         for (int64_t u = s0; u < s1; ++u, ++i) {
           const int kt = static_cast<int>(u % KT);
           const int s = static_cast<int>(i % STAGES);
@@ -986,9 +1162,14 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
           const uint32_t a_base = smem_u32(sA + s * Cfg::A_BYTES);
           const uint32_t b_base = smem_u32(sB + s * Cfg::B_BYTES);
           const uint32_t t_sf = tmem_base + Cfg::TMEM_SF + static_cast<uint32_t>(s) * 32;
-          for (int j = 0; j < na; ++j)
-            mma_mxf4nvf4(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
-                         t_sf + 4 * j, t_sf + 16 + 4 * j, (u != s0 || j != 0) ? 1u : 0u);
+          for (int j = 0; j < na; ++j) {
+            if constexpr (MX)
+              mma_mxf4_block32(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
+                               t_sf + 4 * j, t_sf + 16 + 4 * j, (lora_in || u != s0 || j != 0) ? 1u : 0u);
+            else
+              mma_mxf4nvf4(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j), idesc,
+                           t_sf + 4 * j, t_sf + 16 + 4 * j, (lora_in || u != s0 || j != 0) ? 1u : 0u);
+          }
           tc_commit(&empty[s]);
         }
         if (!ok) break;
@@ -1008,18 +1189,6 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
     const uint32_t quarter = static_cast<uint32_t>(warp & 3);
     const int group = (warp - Cfg::SF_WARP0) >> 2;
     float d6 = 0.0f;
-    if constexpr (QX) {
-      // the activation's per-tensor scale and the 127 decoded scales, as the quantizer builds them
-      const float sg = decode_x_scale(x_gs_in, x_amax);
-      d6 = __fmul_rn(6.0f, sg);
-      const int t = threadIdx.x - Cfg::SF_WARP0 * 32;
-      if (t < 128) {
-        const float eff = __fmul_rn(e4m3_to_float(static_cast<uint32_t>(t)), sg);
-        tab->eff[t] = eff;
-        tab->rcp[t] = eff == 0.0f ? 0.0f : __frcp_rn(eff);
-      }
-      asm volatile("bar.sync 2, %0;" ::"n"(4 * Cfg::SF_GROUPS * 32) : "memory");  // the table is complete
-    }
     // QX work items of a unit for this warp: (row, block) = (it / 4, it % 4) of its
     // K-quarter, it = lane + 32 j over the M rows that exist (at most 4 per lane)
     const int items = QX ? M * 4 : 0;
@@ -1054,6 +1223,18 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
       }
       if (next_u >= 0) load_unit(next_u);
     }
+    if constexpr (QX) {
+      // the activation's per-tensor scale and the 127 decoded scales, as the quantizer builds them
+      const float sg = decode_x_scale(x_gs_in, x_amax);
+      d6 = __fmul_rn(6.0f, sg);
+      const int t = threadIdx.x - Cfg::SF_WARP0 * 32;
+      if (t < 128) {
+        const float eff = __fmul_rn(e4m3_to_float(static_cast<uint32_t>(t)), sg);
+        tab->eff[t] = eff;
+        tab->rcp[t] = eff == 0.0f ? 0.0f : __frcp_rn(eff);
+      }
+      asm volatile("bar.sync 2, %0;" ::"n"(4 * Cfg::SF_GROUPS * 32) : "memory");  // the table is complete
+    }
     bool ok = true;
     for (int sg = 0; ok && decode_segment(sg, u0, u1, KT, s0, s1); ++sg) {
       for (int64_t u = s0; u < s1; ++u, ++i) {
@@ -1080,8 +1261,10 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
             }
             if (nu >= 0) load_unit(nu);
           }
-          // the stage's weight bytes landed, so the MMAs that last read its B tile are done
-          if (!warp_wait(&full[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull + 2)) {
+          // the MMAs of unit i - STAGES are done, so the stage's B tile and TMEM region are
+          // free: the activation is encoded while the unit's weights are still in flight
+          if (!warp_wait(&empty[s], (static_cast<uint32_t>(i / STAGES) & 1u) ^ 1u, abort_flag, status,
+                         kErrWaitFull + 9)) {
             ok = false;
             break;
           }
@@ -1126,6 +1309,11 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
             ok = false;
             break;
           }
+          // the weight scales of the unit landed
+          if (!warp_wait(&full[s], static_cast<uint32_t>(i / STAGES) & 1u, abort_flag, status, kErrWaitFull + 2)) {
+            ok = false;
+            break;
+          }
           const uint8_t* fa = sSFA + s * Cfg::SFA_BYTES + lane * 16;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -1149,16 +1337,20 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
           const uint8_t* fb = sSFB + s * Cfg::SFB_BYTES + lane * 16;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint4 a4 = *reinterpret_cast<const uint4*>(fa + j * Cfg::SF_ATOM);
-            const uint4 b4 = *reinterpret_cast<const uint4*>(fb + j * Cfg::SF_ATOM);
-            v[4 * j] = a4.x;
-            v[4 * j + 1] = a4.y;
-            v[4 * j + 2] = a4.z;
-            v[4 * j + 3] = a4.w;
-            v[16 + 4 * j] = b4.x;
-            v[16 + 4 * j + 1] = b4.y;
-            v[16 + 4 * j + 2] = b4.z;
-            v[16 + 4 * j + 3] = b4.w;
+            // MXFP4: atom j / 2 serves MMAs j and j + 1; MMA j's two block-32 scale bytes
+            // go to the low half of its words (scale-factor id 0)
+            const int sh = MX ? 16 * (j & 1) : 0;
+            const uint32_t keep = MX ? 0xFFFFu : 0xFFFFFFFFu;
+            const uint4 a4 = *reinterpret_cast<const uint4*>(fa + (MX ? (j >> 1) : j) * Cfg::SF_ATOM);
+            const uint4 b4 = *reinterpret_cast<const uint4*>(fb + (MX ? (j >> 1) : j) * Cfg::SF_ATOM);
+            v[4 * j] = (a4.x >> sh) & keep;
+            v[4 * j + 1] = (a4.y >> sh) & keep;
+            v[4 * j + 2] = (a4.z >> sh) & keep;
+            v[4 * j + 3] = (a4.w >> sh) & keep;
+            v[16 + 4 * j] = (b4.x >> sh) & keep;
+            v[16 + 4 * j + 1] = (b4.y >> sh) & keep;
+            v[16 + 4 * j + 2] = (b4.z >> sh) & keep;
+            v[16 + 4 * j + 3] = (b4.w >> sh) & keep;
           }
         }
         tc_fence_after();
@@ -1171,7 +1363,8 @@ __global__ void __launch_bounds__(DecodeCfg<QX>::THREADS)
     }
   } else {
     // ---------------- epilogue (warps 0-3): lane = weight row n, 32 columns = activation rows m ----------------
-    const float alpha = QX ? __fmul_rn(decode_x_scale(x_gs_in, x_amax), *b_gs) : __fmul_rn(*a_gs, *b_gs);
+    const float alpha = MX ? 1.0f  // MXFP4 has no per-tensor scales
+                           : (QX ? __fmul_rn(decode_x_scale(x_gs_in, x_amax), *b_gs) : __fmul_rn(*a_gs, *b_gs));
     int64_t s0, s1;
     for (int q = 0; decode_segment(q, u0, u1, KT, s0, s1); ++q) {
       const int tile = static_cast<int>(s0 / KT);
@@ -1304,29 +1497,33 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
 
 // Swizzled scale buffer of `rows` rows viewed as [row groups][K atoms][128 words]:
 // box = 4 atoms (one K-tile) x `groups` row groups.  Out-of-range atoms/groups read 0.
-bool encode_sf_map(CUtensorMap* map, const uint8_t* sf, int64_t rows, int64_t K, int groups) {
+bool encode_sf_map(CUtensorMap* map, const uint8_t* sf, int64_t rows, int64_t K, int groups, bool mx = false) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const int64_t k_atoms = (K + 63) / 64;
+  // an atom holds 4 scales per row: 64 values of K (NVFP4) or 128 (MXFP4); a K-tile of
+  // 256 values is 4 or 2 atoms
+  const int64_t k_atoms = mx ? (K + 127) / 128 : (K + 63) / 64;
   const int64_t row_groups = (rows + 127) / 128;
   const cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(k_atoms), static_cast<cuuint64_t>(row_groups)};
   const cuuint64_t strides[2] = {512u, static_cast<cuuint64_t>(k_atoms * 512)};
-  const cuuint32_t box[3] = {128u, 4u, static_cast<cuuint32_t>(groups)};
+  const cuuint32_t box[3] = {128u, mx ? 2u : 4u, static_cast<cuuint32_t>(groups)};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(sf), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <bool LR, bool MX>
 int max_pair_clusters(int dev) {
+  using Cfg = PairCfg<LR>;
   static std::once_flag once[64];
   static int clusters[64];
   std::call_once(once[dev & 63], [&] {
     int n = 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 148);
-    cfg.blockDim = dim3(PairCfg::THREADS);
-    cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -1334,10 +1531,12 @@ int max_pair_clusters(int dev) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel, &cfg) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_pair_kernel<LR, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM_BYTES) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<LR, MX>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
       n = 0;
+    }
     clusters[dev & 63] = n;
   });
   return clusters[dev & 63];
@@ -1356,24 +1555,49 @@ bool encode_c_map(CUtensorMap* map, uint16_t* c, int64_t M, int64_t N, int64_t l
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// BF16 rows x R matrix (row stride R elements, R <= 64): box = box_rows x 64 values
+// (one 128-byte row per box row), 128-byte swizzle; values past R and rows past the
+// last read as zero.  The low-rank operands (B's rows, t / alpha).
+bool encode_bf16_rows_map(CUtensorMap* map, const uint16_t* base, int64_t rows, int64_t R, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(R), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(R * 2)};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool LR, bool MX>
 cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
-                        uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream) {
-  CUtensorMap ta, tb, tsa, tsb, tc;
+                        uint16_t* c, int64_t ldc, uint32_t* status, const uint16_t* lora_b, const uint16_t* thi,
+                        const uint16_t* tlo, int64_t rank, cudaStream_t stream) {
+  using Cfg = PairCfg<LR>;
+  CUtensorMap ta, tb, tsa, tsb, tc, tlb, tth, ttl;
   if (!encode_codes_map(&ta, a_codes, M, K, 128) || !encode_codes_map(&tb, b_codes, N, K, 128) ||
-      !encode_sf_map(&tsa, a_sf, M, K, 1) || !encode_sf_map(&tsb, b_sf, N, K, 2) ||
+      !encode_sf_map(&tsa, a_sf, M, K, 1, MX) || !encode_sf_map(&tsb, b_sf, N, K, 2, MX) ||
       !encode_c_map(&tc, c, M, N, ldc))
     return cudaErrorInvalidValue;
+  if (LR) {
+    if (!encode_bf16_rows_map(&tlb, lora_b, N, rank, 128) || !encode_bf16_rows_map(&tth, thi, M, rank, 128) ||
+        !encode_bf16_rows_map(&ttl, tlo, M, rank, 128))
+      return cudaErrorInvalidValue;
+  } else {
+    tlb = tth = ttl = tc;  // unused slots
+  }
   int dev = 0;
   cudaGetDevice(&dev);
-  const int max_clusters = max_pair_clusters(dev);
+  const int max_clusters = max_pair_clusters<LR, MX>(dev);
   if (max_clusters <= 0) return cudaErrorLaunchOutOfResources;
   const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
   const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
-  cfg.blockDim = dim3(PairCfg::THREADS);
-  cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1383,8 +1607,8 @@ cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float
   set_programmatic(attr[1]);
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tb, tsa, tsb, tc, a_gs, b_gs, static_cast<int>(M),
-                            static_cast<int>(N), static_cast<int>(K), status);
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<LR, MX>, ta, tb, tsa, tsb, tc, tlb, tth, ttl, static_cast<int>(rank), c,
+                            ldc, a_gs, b_gs, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), status);
 }
 
 // CTAs of the decode kernel: one per weight tile when the tiles number between 70 %
@@ -1399,21 +1623,22 @@ int64_t decode_grid(int64_t N, int64_t K, int sms) {
 // Launch the decode kernel: QX = false reads the activation's codes and scales
 // (tmap_x over a_codes, a_sf, a_gs); QX = true quantizes the BF16 activation x (row
 // stride ld_x) itself, global scale from x_gs_in or the amax word x_amax.
-template <bool QX>
-cudaError_t launch_decode(const CUtensorMap& tw, const CUtensorMap& tx, const uint8_t* a_sf, const float* a_gs,
+template <bool QX, bool LR, bool MX = false>
+cudaError_t launch_decode(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& tlb, const CUtensorMap& tthi,
+                          const CUtensorMap& ttlo, int rank, const uint8_t* a_sf, const float* a_gs,
                           const uint16_t* x, int64_t ld_x, const float* x_gs_in, const uint32_t* x_amax, int64_t M,
                           const uint8_t* b_sf,
                           const float* b_gs, int64_t N, int64_t K, uint16_t* c, int64_t ldc, uint32_t* status,
                           uint8_t* scratch, cudaStream_t stream) {
-  using Cfg = DecodeCfg<QX>;
+  using Cfg = DecodeCfg<QX, LR>;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   std::call_once(once[dev & 63], [&] {
-    attr_err[dev & 63] = cudaFuncSetAttribute(gemm_decode_kernel<QX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              Cfg::SMEM_BYTES);
+    attr_err[dev & 63] = cudaFuncSetAttribute(gemm_decode_kernel<QX, LR, MX>,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   });
   if (attr_err[dev & 63] != cudaSuccess) return attr_err[dev & 63];
   const int64_t KT = (K + 255) / 256;
@@ -1432,9 +1657,9 @@ cudaError_t launch_decode(const CUtensorMap& tw, const CUtensorMap& tx, const ui
   set_programmatic(attr[0]);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_decode_kernel<QX>, tw, tx, b_sf, a_sf, a_gs, b_gs, x, ld_x, x_gs_in, x_amax,
-                            c, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), ldc, max_seg, partial,
-                            counters, status);
+  return cudaLaunchKernelEx(&cfg, gemm_decode_kernel<QX, LR, MX>, tw, tx, tlb, tthi, ttlo, rank, b_sf, a_sf, a_gs, b_gs,
+                            x, ld_x, x_gs_in, x_amax, c, static_cast<int>(M), static_cast<int>(N),
+                            static_cast<int>(K), ldc, max_seg, partial, counters, status);
 }
 
 template <int BN>
@@ -1496,11 +1721,12 @@ cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
     CUtensorMap tw, tx;
     if (!encode_codes_map(&tw, b_codes, N, K, 128) || !encode_codes_map(&tx, a_codes, M, K, DecodeCfg<false>::BN))
       return cudaErrorInvalidValue;
-    return launch_decode<false>(tw, tx, a_sf, a_gs, nullptr, 0, nullptr, nullptr, M, b_sf, b_gs, N, K, c, ldc, status,
-                                reinterpret_cast<uint8_t*>(status) + 256, stream);
+    return launch_decode<false, false>(tw, tx, tw, tw, tw, 0, a_sf, a_gs, nullptr, 0, nullptr, nullptr, M, b_sf, b_gs,
+                                       N, K, c, ldc, status, reinterpret_cast<uint8_t*>(status) + 256, stream);
   }
   if (M > 128 && N > 128)
-    return launch_pair(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status, stream);
+    return launch_pair<false, false>(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status, nullptr, nullptr,
+                              nullptr, 0, stream);
   const int bn = N > 128 ? 256 : 128;
   CUtensorMap ta, tb;
   if (!encode_codes_map(&ta, a_codes, M, K, 128) || !encode_codes_map(&tb, b_codes, N, K, bn))
@@ -1515,9 +1741,46 @@ cudaError_t launch_decode_quantize_x(const uint16_t* x, int64_t M, int64_t K, in
                                      uint8_t* scratch, cudaStream_t stream) {
   CUtensorMap tw;
   if (!encode_codes_map(&tw, b_codes, N, K, 128)) return cudaErrorInvalidValue;
-  // (the activation is read with plain loads; the second tensor-map slot is unused)
-  return launch_decode<true>(tw, tw, nullptr, nullptr, x, ld_x, x_gs_in, x_amax, M, b_sf, b_gs, N, K, c, ldc, status,
-                             scratch, stream);
+  // (the activation is read with plain loads; the unused tensor-map slots repeat tw)
+  return launch_decode<true, false>(tw, tw, tw, tw, tw, 0, nullptr, nullptr, x, ld_x, x_gs_in, x_amax, M, b_sf, b_gs,
+                                    N, K, c, ldc, status, scratch, stream);
+}
+
+cudaError_t launch_gemm_mx(const uint8_t* a_codes, const uint8_t* a_sf, int64_t M, const uint8_t* b_codes,
+                           const uint8_t* b_sf, int64_t N, int64_t K, uint16_t* c, int64_t ldc, uint32_t* status,
+                           cudaStream_t stream) {
+  if (M <= DecodeCfg<false>::BN) {
+    CUtensorMap tw, tx;
+    if (!encode_codes_map(&tw, b_codes, N, K, 128) || !encode_codes_map(&tx, a_codes, M, K, DecodeCfg<false>::BN))
+      return cudaErrorInvalidValue;
+    return launch_decode<false, false, true>(tw, tx, tw, tw, tw, 0, a_sf, nullptr, nullptr, 0, nullptr, nullptr, M,
+                                             b_sf, nullptr, N, K, c, ldc, status,
+                                             reinterpret_cast<uint8_t*>(status) + 256, stream);
+  }
+  return launch_pair<false, true>(a_codes, a_sf, nullptr, M, b_codes, b_sf, nullptr, N, K, c, ldc, status, nullptr,
+                                  nullptr, nullptr, 0, stream);
+}
+
+cudaError_t launch_gemm_lora(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
+                             const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
+                             uint16_t* c, int64_t ldc, uint32_t* status, const uint16_t* lora_b, const uint16_t* thi,
+                             const uint16_t* tlo, int64_t R, cudaStream_t stream) {
+  return launch_pair<true, false>(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status, lora_b, thi, tlo, R,
+                           stream);
+}
+
+cudaError_t launch_decode_quantize_x_lora(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x,
+                                          const float* x_gs_in, const uint32_t* x_amax, const uint8_t* b_codes,
+                                          const uint8_t* b_sf, const float* b_gs, int64_t N, const uint16_t* lora_b,
+                                          const uint16_t* thi, const uint16_t* tlo, int64_t R, uint16_t* c,
+                                          int64_t ldc, uint32_t* status, uint8_t* scratch, cudaStream_t stream) {
+  CUtensorMap tw, tlb, tth, ttl;
+  if (!encode_codes_map(&tw, b_codes, N, K, 128) || !encode_bf16_rows_map(&tlb, lora_b, N, R, 128) ||
+      !encode_bf16_rows_map(&tth, thi, M, R, DecodeCfg<true, true>::BN) ||
+      !encode_bf16_rows_map(&ttl, tlo, M, R, DecodeCfg<true, true>::BN))
+    return cudaErrorInvalidValue;
+  return launch_decode<true, true>(tw, tw, tlb, tth, ttl, static_cast<int>(R), nullptr, nullptr, x, ld_x, x_gs_in,
+                                   x_amax, M, b_sf, b_gs, N, K, c, ldc, status, scratch, stream);
 }
 
 }  // namespace nvfp4

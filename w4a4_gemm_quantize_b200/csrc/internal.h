@@ -25,6 +25,13 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, bool swizzled, const float* gs,
                               int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out, cudaStream_t stream);
 
+// MXFP4 quantizer and reconstruction (quantize.cu): blocks of 32, E8M0 scales (the
+// swizzled layout has the same 128 x 4 atoms, one byte per 32-value block).
+cudaError_t launch_quantize_mx(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, bool swizzled,
+                               uint8_t* codes, uint8_t* scales, cudaStream_t stream);
+cudaError_t launch_dequantize_mx(const uint8_t* codes, const uint8_t* scales, bool swizzled, int64_t rows,
+                                 int64_t cols, uint16_t* out, int64_t ld_out, cudaStream_t stream);
+
 // Bounded-wait self test (quantize.cu).
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t stream);
 
@@ -42,6 +49,38 @@ cudaError_t launch_decode_quantize_x(const uint16_t* x, int64_t M, int64_t K, in
                                      const uint32_t* x_amax, const uint8_t* b_codes, const uint8_t* b_sf,
                                      const float* b_gs, int64_t N, uint16_t* c, int64_t ldc, uint32_t* status,
                                      uint8_t* scratch, cudaStream_t stream);
+
+// The same with the low-rank branch added to the accumulator: lora_b (N x R BF16) and
+// t / alpha as BF16 hi and lo parts (M x R each, from launch_lora_down), R <= 64.
+cudaError_t launch_decode_quantize_x_lora(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x,
+                                          const float* x_gs_in, const uint32_t* x_amax, const uint8_t* b_codes,
+                                          const uint8_t* b_sf, const float* b_gs, int64_t N, const uint16_t* lora_b,
+                                          const uint16_t* thi, const uint16_t* tlo, int64_t R, uint16_t* c,
+                                          int64_t ldc, uint32_t* status, uint8_t* scratch, cudaStream_t stream);
+
+// The MXFP4 GEMM C = A B^T (E8M0 block-32 scales, swizzled, no per-tensor scales):
+// the small-M kernel for M <= 32 (workspace as nvfp4_gemm's), the CTA-pair kernel above.
+cudaError_t launch_gemm_mx(const uint8_t* a_codes, const uint8_t* a_sf, int64_t M, const uint8_t* b_codes,
+                           const uint8_t* b_sf, int64_t N, int64_t K, uint16_t* c, int64_t ldc, uint32_t* status,
+                           cudaStream_t stream);
+
+// The CTA-pair GEMM (any M, N; meant for M > 32) with the low-rank branch: lora_b
+// (N x R BF16) and t / alpha as BF16 hi and lo parts (M x R each), R <= 64.
+cudaError_t launch_gemm_lora(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
+                             const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
+                             uint16_t* c, int64_t ldc, uint32_t* status, const uint16_t* lora_b, const uint16_t* thi,
+                             const uint16_t* tlo, int64_t R, cudaStream_t stream);
+
+// The low-rank down-projection t = BF16(x A^T) (x M x K, A R x K BF16, R % 16 == 0,
+// R <= 64), with t / alpha as BF16 hi and lo parts (alpha = s_gA s_gB, s_gA from
+// x_gs_in or the amax word x_amax); t_out may be null.  counters: lora_counter_bytes(M)
+// zeroed bytes (left zeroed); partial: lora_partial_bytes(M, K, R) bytes.
+cudaError_t launch_lora_down(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x, const float* x_gs_in,
+                             const uint32_t* x_amax, const float* w_gs, const uint16_t* lora_a, int64_t R,
+                             uint16_t* t_out, uint16_t* thi, uint16_t* tlo, uint32_t* counters, float* partial,
+                             uint32_t* status, cudaStream_t stream);
+size_t lora_partial_bytes(int64_t M, int64_t K, int64_t R);
+size_t lora_counter_bytes(int64_t M);
 
 // Bytes the GEMM needs in its workspace after the 256-byte status block
 // (split-K partial tiles of the small-M kernel); 0 when none.

@@ -305,6 +305,118 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const uint8_t* __r
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// MXFP4: blocks of 32 values along the row, an E8M0 (power-of-two) scale per block, no
+// per-tensor scale -- the OCP Microscaling Formats (MX) v1.0 rule, the outside reading
+// for the format that "Cuantización en Producción: AWQ, GPTQ, GGUF K-quants, FP8,
+// MXFP4/NVFP4" names without its block size or scale type: shared = floor(log2 amax)
+// - 2 clamped to [-127, 127], scale byte shared + 127 (0 for an all-zero block), codes
+// = E2M1_sat(x * 2^-shared) (RNE, the sign kept).
+// ---------------------------------------------------------------------------------------------
+
+// floor(log2 a) of a positive finite float from its bits (subnormals included).
+__device__ __forceinline__ int floor_log2_bits(uint32_t bits) {
+  const int e = static_cast<int>(bits >> 23);
+  if (e > 0) return e - 127;
+  return (31 - __clz(static_cast<int>(bits & 0x7FFFFFu))) - 149;
+}
+
+// 2^k as a float for k in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float pow2f(int k) {
+  return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// One thread per 32-value block, one warp per 32 consecutive blocks of a row.
+template <bool SWZ>
+__global__ void __launch_bounds__(kThreads) quantize_mx_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                               int64_t cols, int64_t ld, uint8_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ scales) {
+  grid_dependency_wait();
+  const int64_t nblk = cols / 32;
+  const int64_t atoms_per_group = (nblk + 3) / 4;
+  const int64_t chunks = (nblk + 31) / 32;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (int64_t task = w; task < rows * chunks; task += nwarps) {
+    const int64_t r = task / chunks, cb = (task - r * chunks) * 32 + lane;
+    const bool active = cb < nblk;
+    uint32_t sbyte = 0;
+    if (active) {
+      const uint16_t* src = x + r * ld + cb * 32;
+      uint4 v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = ld_nc_v4(src + 8 * i);
+      uint32_t m = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m = vmax_mag(m, v[i]);
+      const uint32_t amax_bits = max(m & 0xFFFFu, m >> 16) << 16;
+      int shared = amax_bits == 0 ? -127 : floor_log2_bits(amax_bits) - 2;
+      shared = max(-127, min(127, shared));
+      sbyte = static_cast<uint32_t>(shared + 127);
+      const float inv = pow2f(-shared);
+      uint32_t out[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {  // eight values per 32-bit word of codes
+        const uint4 q = v[h];
+        const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+        float y[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          y[2 * k] = __fmul_rn(__uint_as_float(wd[k] << 16), inv);
+          y[2 * k + 1] = __fmul_rn(__uint_as_float(wd[k] & 0xFFFF0000u), inv);
+        }
+        out[h] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+      }
+      *reinterpret_cast<uint4*>(codes + r * (cols / 2) + cb * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+      if (!SWZ) scales[r * nblk + cb] = static_cast<uint8_t>(sbyte);
+    }
+    if (SWZ) {
+      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sbyte, 1);
+      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sbyte, 2);
+      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sbyte, 3);
+      if (active && (lane & 3) == 0) {
+        const int64_t off = ((r >> 7) * atoms_per_group + (cb >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+        *reinterpret_cast<uint32_t*>(scales + off) = sbyte | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      }
+    }
+  }
+  if (SWZ) zero_scale_padding(scales, rows, nblk);
+}
+
+// BF16 reconstruction q * 2^(s - 127), one thread per 32-value block.
+template <bool SWZ>
+__global__ void __launch_bounds__(kThreads) dequantize_mx_kernel(const uint8_t* __restrict__ codes,
+                                                                 const uint8_t* __restrict__ scales, int64_t rows,
+                                                                 int64_t cols, uint16_t* __restrict__ out,
+                                                                 int64_t ld_out) {
+  grid_dependency_wait();
+  const int64_t nblk = cols / 32;
+  const int64_t atoms_per_group = (nblk + 3) / 4;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < rows * nblk; b += stride) {
+    const int64_t r = b / nblk, cb = b - r * nblk;
+    const uint4 cw = *reinterpret_cast<const uint4*>(codes + r * (cols / 2) + cb * 16);
+    const uint32_t s = SWZ ? scales[swizzled_offset(r, cb, atoms_per_group)] : scales[b];
+    const float scale = pow2f(static_cast<int>(s) - 127);
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+    uint4* dst = reinterpret_cast<uint4*>(out + r * ld_out + cb * 32);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t h2 = e2m1x2_to_half2(words[h], k);
+        const float q_lo = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFFu)));
+        const float q_hi = __half2float(__ushort_as_half(static_cast<uint16_t>(h2 >> 16)));
+        o[k] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(q_lo, scale)))) |
+               (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(q_hi, scale)))) << 16);
+      }
+      dst[h] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 // One thread waits, with the kernels' bounded wait, on an mbarrier that nothing
 // completes; it gives up after timeout_ns and records kErrSelfTest.
 __global__ void selftest_wait_kernel(uint32_t* status, uint64_t timeout_ns) {
@@ -371,6 +483,42 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64
   else
     e = swizzled ? NVFP4_Q(0, true) : NVFP4_Q(0, false);
 #undef NVFP4_Q
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_quantize_mx(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, bool swizzled,
+                               uint8_t* codes, uint8_t* scales, cudaStream_t stream) {
+  const int64_t nblk = cols / 32;
+  const int64_t pads = swizzled ? ((rows + 127) / 128 * 128) * ((nblk + 3) / 4 * 4) - rows * nblk : 0;
+  const int64_t work = rows * ((nblk + 31) / 32) * 32;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid_for(work > pads ? work : pads, kThreads));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = swizzled ? cudaLaunchKernelEx(&cfg, quantize_mx_kernel<true>, x, rows, cols, ld, codes, scales)
+                                 : cudaLaunchKernelEx(&cfg, quantize_mx_kernel<false>, x, rows, cols, ld, codes, scales);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_dequantize_mx(const uint8_t* codes, const uint8_t* scales, bool swizzled, int64_t rows,
+                                 int64_t cols, uint16_t* out, int64_t ld_out, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid_for(rows * (cols / 32), kThreads));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e =
+      swizzled ? cudaLaunchKernelEx(&cfg, dequantize_mx_kernel<true>, codes, scales, rows, cols, out, ld_out)
+               : cudaLaunchKernelEx(&cfg, dequantize_mx_kernel<false>, codes, scales, rows, cols, out, ld_out);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
