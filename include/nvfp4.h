@@ -147,10 +147,10 @@ nvfp4_status nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const f
                         const float *b_global_scale, int64_t N, int64_t K, void *c, int64_t ldc,
                         void *workspace, size_t workspace_bytes, void *stream);
 
-/* Workspace nvfp4_linear needs (device memory, any content on entry): 512 bytes
- * (status word, the activation's amax and global scale), plus for M <= 32 the
- * small-M kernel's tile counters and partial tiles, for M > 32 the activation's
- * codes and swizzled scales. */
+/* Workspace nvfp4_linear and nvfp4_linear_fused need (device memory, any content
+ * on entry): 512 bytes (status word, the activation's amax and global scale), for
+ * M <= 32 the small-M kernel's tile counters and partial tiles, then the
+ * activation's codes and swizzled scales. */
 size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* The W4A4 linear layer: the BF16 activation X is quantized on this call (absmax
@@ -158,9 +158,7 @@ size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * -- the page "NVFP4 en difusión: la misma cuantización, un motor completamente
  * distinto", section 2 "NVFP4 sin vLLM: torch._scaled_mm a mano" (the activation
  * is quantized on every forward, 16-block by 16-block, while the weights come
- * quantized from the checkpoint; out = (A s_a)(B s_b)^T in BF16), with the
- * quantization done in the same kernel as the matmul where the activation is small,
- * as section 3 describes for nunchaku's fused kernel.
+ * quantized from the checkpoint; out = (A s_a)(B s_b)^T in BF16).
  *   x            device, BF16, M x K, row stride ld_x elements (ld_x >= K, ld_x % 8 == 0).
  *   x_global_scale  device float or NULL: the activation's per-tensor FP32 scale.
  *                Given (a calibrated activation scale: "Tu pipeline NVFP4 ...",
@@ -174,16 +172,30 @@ size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   c            device BF16, M x N, row stride ldc (ldc >= N, ldc % 8 == 0).
  *   M, N >= 1; K >= 32, K % 32 == 0.
  * The result equals nvfp4_quantize(x, ABSMAX, SWIZZLED, x_global_scale) followed by
- * nvfp4_gemm bit for bit.  For M <= 32 one kernel quantizes the activation K-tiles
- * it consumes and multiplies (plus the amax pass when x_global_scale is NULL); for
- * M > 32 the quantizer writes the activation's codes into the workspace and the
- * GEMM reads them (kernels chained with programmatic dependent launch).
+ * nvfp4_gemm bit for bit, and that is what runs: one memset of the workspace's
+ * counters, the amax pass (x_global_scale NULL), the quantizer writing the
+ * activation's codes into the workspace and the GEMM, chained with programmatic
+ * dependent launch (the small-M GEMM starts its weight stream before the quantizer
+ * has finished).
  * Errors: INVALID_ARG, SHAPE, ALIGNMENT, WORKSPACE, UNSUPPORTED_DEVICE, CUDA; a
  * device-side timeout is read with nvfp4_read_device_error(workspace, ...). */
 nvfp4_status nvfp4_linear(const void *x, int64_t M, int64_t K, int64_t ld_x, const float *x_global_scale,
                           const uint8_t *w_codes, const uint8_t *w_scales, const float *w_global_scale,
                           int64_t N, void *c, int64_t ldc, void *workspace, size_t workspace_bytes,
                           void *stream);
+
+/* nvfp4_linear for M <= 32 with the quantization inside the GEMM kernel, as the same
+ * page's section 3 describes for nunchaku's fused kernel: every CTA quantizes the
+ * activation K-tiles it consumes (absmax, the quantizer's arithmetic) instead of
+ * reading codes a separate pass wrote.  Same arguments, workspace
+ * (nvfp4_linear_workspace_bytes) and result bit for bit as nvfp4_linear; M > 32
+ * returns SHAPE.  Every CTA of the small-M GEMM needs the whole activation, so each
+ * quantizes all of it: on B200 this is slower than nvfp4_linear for the shapes
+ * measured (decode M = 1, 8, 32 against a 14336 x 4096 weight). */
+nvfp4_status nvfp4_linear_fused(const void *x, int64_t M, int64_t K, int64_t ld_x, const float *x_global_scale,
+                                const uint8_t *w_codes, const uint8_t *w_scales, const float *w_global_scale,
+                                int64_t N, void *c, int64_t ldc, void *workspace, size_t workspace_bytes,
+                                void *stream);
 
 /* Workspace nvfp4_linear_lora needs (device memory, any content on entry). */
 size_t nvfp4_linear_lora_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t R);

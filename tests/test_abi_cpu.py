@@ -192,13 +192,15 @@ def test_noalloc_validation_before_any_cuda_call(lib):
     assert q() in (4, 5)
 
 
-def test_linear_validation_before_any_cuda_call(lib):
+@pytest.mark.parametrize("entry", ["nvfp4_linear", "nvfp4_linear_fused"])
+def test_linear_validation_before_any_cuda_call(lib, entry):
     P = ctypes.c_void_p
+    fn = getattr(lib, entry)
 
     def g(M=8, N=256, K=64, ld=64, ldc=256, ptr=16, ws=16, ws_bytes=1 << 30, x_gs=None):
         p = P(ptr) if ptr else None
-        return lib.nvfp4_linear(p, M, K, ld, P(x_gs) if x_gs else None, p, p, P(16), N, p, ldc,
-                                P(ws) if ws else None, ws_bytes, None)
+        return fn(p, M, K, ld, P(x_gs) if x_gs else None, p, p, P(16), N, p, ldc, P(ws) if ws else None, ws_bytes,
+                  None)
 
     assert g(K=48, ld=48) == 2          # K % 32
     assert g(M=0) == 1
@@ -209,7 +211,16 @@ def test_linear_validation_before_any_cuda_call(lib):
     assert g(ptr=8) == 3
     assert g(x_gs=18) == 3
     assert g() in (4, 5)
-    assert lib.nvfp4_linear_workspace_bytes(8, 14336, 4096) == 512 + lib.nvfp4_gemm_workspace_bytes(8, 14336, 4096) - 256
+    if entry == "nvfp4_linear_fused":
+        assert g(M=33) == 2             # the fused kernel is the small-M one
+
+
+def test_linear_workspace_layout(lib):
+    # header, the small-M GEMM's counters and partial tiles, the activation's codes and scales
+    for M in (8, 32):
+        gemm_scratch = lib.nvfp4_gemm_workspace_bytes(M, 14336, 4096) - 256
+        act = -(-(M * 2048) // 256) * 256 + lib.nvfp4_scales_bytes(M, 4096, 0)
+        assert lib.nvfp4_linear_workspace_bytes(M, 14336, 4096) >= 512 + gemm_scratch + act
     assert lib.nvfp4_linear_workspace_bytes(4096, 14336, 4096) >= 512 + 4096 * 2048 + 4096 * 256
 
 

@@ -53,6 +53,7 @@ SIGNATURES = {
     "nvfp4_gemm": ([_P, _P, _P, _I64, _P, _P, _P, _I64, _I64, _P, _I64, _P, _SZ, _P], _I),
     "nvfp4_linear_workspace_bytes": ([_I64, _I64, _I64], _SZ),
     "nvfp4_linear": ([_P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, _P, _I64, _P, _SZ, _P], _I),
+    "nvfp4_linear_fused": ([_P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, _P, _I64, _P, _SZ, _P], _I),
     "nvfp4_linear_lora_workspace_bytes": ([_I64, _I64, _I64, _I64], _SZ),
     "nvfp4_linear_lora": ([_P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, _P, _P, _I64, _P, _I64, _P, _P, _SZ, _P], _I),
     "mxfp4_scales_bytes": ([_I64, _I64, _I], _SZ),
@@ -236,11 +237,14 @@ def last_launch_count() -> int:
 
 
 def linear(x: torch.Tensor, w: NVFP4Tensor, x_global_scale: Optional[torch.Tensor] = None,
-           out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+           out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None,
+           fused: bool = False) -> torch.Tensor:
     """W4A4 linear layer C = Q(x) w^T in BF16: the activation x (M x K BF16) is
     quantized on this call with absmax block scales -- under `x_global_scale` (a
     device float, e.g. a calibrated activation scale) or, if None, amax(|x|)/2688
-    computed on the device -- and multiplied by the pre-quantized weight w (N x K)."""
+    computed on the device -- and multiplied by the pre-quantized weight w (N x K).
+    fused=True (M <= 32) quantizes the activation inside the GEMM kernel
+    (nvfp4_linear_fused); the result is the same bit for bit."""
     lib = load_library()
     if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda or x.stride(1) != 1:
         raise ValueError("x must be a 2-D row-major bfloat16 CUDA tensor")
@@ -252,10 +256,10 @@ def linear(x: torch.Tensor, w: NVFP4Tensor, x_global_scale: Optional[torch.Tenso
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
         workspace = torch.empty(lib.nvfp4_linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=x.device)
-    st = lib.nvfp4_linear(_ptr(x), M, K, x.stride(0), _ptr(x_global_scale), _ptr(w.codes), _ptr(w.scales),
-                          _ptr(w.global_scale), N, _ptr(out), out.stride(0), _ptr(workspace), workspace.numel(),
-                          _stream(stream))
-    _check(st, "nvfp4_linear")
+    fn = lib.nvfp4_linear_fused if fused else lib.nvfp4_linear
+    st = fn(_ptr(x), M, K, x.stride(0), _ptr(x_global_scale), _ptr(w.codes), _ptr(w.scales),
+            _ptr(w.global_scale), N, _ptr(out), out.stride(0), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "nvfp4_linear_fused" if fused else "nvfp4_linear")
     return out
 
 

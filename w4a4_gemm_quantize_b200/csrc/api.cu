@@ -207,64 +207,121 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const f
   return st;
 }
 
+namespace {
+
+// Workspace of nvfp4_linear: the 512-byte header (status word, amax word, the
+// activation's global scale), for M <= 32 the small-M GEMM's counters and partial
+// tiles, then the activation's codes and swizzled scales.  The memset clears the
+// header and the counters (the `zero` bytes).
+struct LinearLayout {
+  size_t gemm_scratch, x_codes, x_scales, zero, total;
+};
+
+LinearLayout linear_layout(int64_t M, int64_t N, int64_t K) {
+  LinearLayout l{};
+  l.gemm_scratch = kLinearHeader;
+  const size_t scratch = M <= 32 ? nvfp4::gemm_scratch_bytes(M, N, K) : 0;
+  l.zero = M <= 32 ? kLinearHeader + (nvfp4::gemm_zero_bytes(M, N, K) - 256) : kLinearHeader;
+  l.x_codes = (kLinearHeader + scratch + 255) / 256 * 256;
+  l.x_scales = l.x_codes + linear_codes_bytes(M, K);
+  l.total = l.x_scales + nvfp4_scales_bytes(M, K, NVFP4_SF_SWIZZLED);
+  return l;
+}
+
+nvfp4_status validate_linear(const void* x, int64_t M, int64_t K, int64_t ld_x, const float* x_global_scale,
+                             const uint8_t* w_codes, const uint8_t* w_scales, const float* w_global_scale, int64_t N,
+                             void* c, int64_t ldc, void* workspace, size_t workspace_bytes, size_t need) {
+  if (M < 1 || N < 1 || K < 1 || ld_x < K || ldc < N) return NVFP4_ERR_INVALID_ARG;
+  if (K % 32 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return NVFP4_ERR_SHAPE;
+  if (!x || !w_codes || !w_scales || !w_global_scale || !c) return NVFP4_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < need) return NVFP4_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(c) || !aligned16(workspace) ||
+      ld_x % 8 != 0 || ldc % 8 != 0 || (reinterpret_cast<uintptr_t>(w_global_scale) & 3u) ||
+      (x_global_scale && (reinterpret_cast<uintptr_t>(x_global_scale) & 3u)))
+    return NVFP4_ERR_ALIGNMENT;
+  return check_device_cached();
+}
+
+}  // namespace
+
 size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 1) return kLinearHeader;
-  if (M <= 32) return kLinearHeader + nvfp4::gemm_scratch_bytes(M, N, K);
-  return kLinearHeader + linear_codes_bytes(M, K) + nvfp4_scales_bytes(M, K, NVFP4_SF_SWIZZLED);
+  return linear_layout(M, N, K).total;
 }
 
 nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, int64_t ld_x, const float* x_global_scale,
                           const uint8_t* w_codes, const uint8_t* w_scales, const float* w_global_scale, int64_t N,
                           void* c, int64_t ldc, void* workspace, size_t workspace_bytes, void* stream) {
   nvfp4::g_last_launches = 0;
-  if (M < 1 || N < 1 || K < 1 || ld_x < K || ldc < N) return NVFP4_ERR_INVALID_ARG;
-  if (K % 32 != 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return NVFP4_ERR_SHAPE;
-  if (!x || !w_codes || !w_scales || !w_global_scale || !c) return NVFP4_ERR_INVALID_ARG;
-  if (!workspace || workspace_bytes < nvfp4_linear_workspace_bytes(M, N, K)) return NVFP4_ERR_WORKSPACE;
-  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(c) || !aligned16(workspace) ||
-      ld_x % 8 != 0 || ldc % 8 != 0 || (reinterpret_cast<uintptr_t>(w_global_scale) & 3u) ||
-      (x_global_scale && (reinterpret_cast<uintptr_t>(x_global_scale) & 3u)))
-    return NVFP4_ERR_ALIGNMENT;
-  nvfp4_status st = check_device_cached();
+  nvfp4_status st = validate_linear(x, M, K, ld_x, x_global_scale, w_codes, w_scales, w_global_scale, N, c, ldc,
+                                    workspace, workspace_bytes,
+                                    M >= 1 && N >= 1 && K >= 1 ? nvfp4_linear_workspace_bytes(M, N, K) : 0);
   if (st != NVFP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const LinearLayout l = linear_layout(M, N, K);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   uint32_t* amax_word = reinterpret_cast<uint32_t*>(ws + 256);
   const uint16_t* xb = static_cast<const uint16_t*>(x);
-  // one memset: the status word, the amax word and (small M) the tile counters
-  const size_t zero = M <= 32 ? kLinearHeader + (nvfp4::gemm_zero_bytes(M, N, K) - 256) : kLinearHeader;
-  if (cudaMemsetAsync(ws, 0, zero, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  // one memset ahead of the chain: the status word, the amax word and (small M) the
+  // tile counters, so that the kernels after it follow one another with programmatic
+  // dependent launch
+  if (cudaMemsetAsync(ws, 0, l.zero, s) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (x_global_scale == nullptr) {
     st = from_cuda(nvfp4::launch_amax(xb, M, K, ld_x, amax_word, s));
     if (st != NVFP4_OK) return st;
     ++nvfp4::g_last_launches;
   }
-  if (M <= 32) {
-    const cudaError_t e = nvfp4::launch_decode_quantize_x(
-        xb, M, K, ld_x, x_global_scale, x_global_scale ? nullptr : amax_word, w_codes, w_scales, w_global_scale, N,
-        static_cast<uint16_t*>(c), ldc, status, ws + kLinearHeader, s);
-    st = from_cuda(e);
-    if (st == NVFP4_OK) ++nvfp4::g_last_launches;
-    return st;
-  }
-  uint8_t* a_codes = ws + kLinearHeader;
-  uint8_t* a_scales = a_codes + linear_codes_bytes(M, K);
+  uint8_t* a_codes = ws + l.x_codes;
+  uint8_t* a_scales = ws + l.x_scales;
   float* a_gs = x_global_scale ? nullptr : reinterpret_cast<float*>(ws + 260);
   st = from_cuda(nvfp4::launch_quantize(xb, M, K, ld_x, NVFP4_SCALE_ABSMAX, true, x_global_scale, amax_word, a_codes,
                                         a_scales, a_gs, nullptr, s));
   if (st != NVFP4_OK) return st;
   ++nvfp4::g_last_launches;
   st = from_cuda(nvfp4::launch_gemm(a_codes, a_scales, x_global_scale ? x_global_scale : a_gs, M, w_codes, w_scales,
-                                    w_global_scale, N, K, static_cast<uint16_t*>(c), ldc, status, s));
+                                    w_global_scale, N, K, static_cast<uint16_t*>(c), ldc, status, s,
+                                    ws + l.gemm_scratch));
   if (st == NVFP4_OK) ++nvfp4::g_last_launches;
   return st;
 }
 
+nvfp4_status nvfp4_linear_fused(const void* x, int64_t M, int64_t K, int64_t ld_x, const float* x_global_scale,
+                                const uint8_t* w_codes, const uint8_t* w_scales, const float* w_global_scale,
+                                int64_t N, void* c, int64_t ldc, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  nvfp4::g_last_launches = 0;
+  if (M > 32) return NVFP4_ERR_SHAPE;
+  nvfp4_status st = validate_linear(x, M, K, ld_x, x_global_scale, w_codes, w_scales, w_global_scale, N, c, ldc,
+                                    workspace, workspace_bytes,
+                                    M >= 1 && N >= 1 && K >= 1 ? nvfp4_linear_workspace_bytes(M, N, K) : 0);
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const LinearLayout l = linear_layout(M, N, K);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  uint32_t* amax_word = reinterpret_cast<uint32_t*>(ws + 256);
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  if (cudaMemsetAsync(ws, 0, l.zero, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (x_global_scale == nullptr) {
+    st = from_cuda(nvfp4::launch_amax(xb, M, K, ld_x, amax_word, s));
+    if (st != NVFP4_OK) return st;
+    ++nvfp4::g_last_launches;
+  }
+  st = from_cuda(nvfp4::launch_decode_quantize_x(xb, M, K, ld_x, x_global_scale,
+                                                 x_global_scale ? nullptr : amax_word, w_codes, w_scales,
+                                                 w_global_scale, N, static_cast<uint16_t*>(c), ldc, status,
+                                                 ws + l.gemm_scratch, s));
+  if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+  return st;
+}
+
+namespace {
+
 // Workspace of nvfp4_linear_lora: the 512-byte header of nvfp4_linear, the
-// down-projection's counters, the small-M kernel's counters (one zeroed range), then
-// the down-projection's partial tiles, t / alpha hi and lo, and the GEMM's scratch
-// (small M) or the activation's codes and scales (large M).
+// down-projection's counters, the small-M kernel's counters (one zeroed range) and
+// partial tiles, then the down-projection's partial tiles, t / alpha hi and lo, and
+// the activation's codes and scales.
 struct LoraLayout {
   size_t lora_counters, gemm_scratch, lora_partial, thi, tlo, x_codes, x_scales, zero, total;
 };
@@ -285,15 +342,15 @@ LoraLayout lora_layout(int64_t M, int64_t N, int64_t K, int64_t R) {
   off = up(off + static_cast<size_t>(M * R * 2));
   l.tlo = off;
   off = up(off + static_cast<size_t>(M * R * 2));
-  if (M > 32) {
-    l.x_codes = off;
-    off += linear_codes_bytes(M, K);
-    l.x_scales = off;
-    off += nvfp4_scales_bytes(M, K, NVFP4_SF_SWIZZLED);
-  }
+  l.x_codes = off;
+  off += linear_codes_bytes(M, K);
+  l.x_scales = off;
+  off += nvfp4_scales_bytes(M, K, NVFP4_SF_SWIZZLED);
   l.total = off;
   return l;
 }
+
+}  // namespace
 
 size_t nvfp4_linear_lora_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t R) {
   if (M < 1 || N < 1 || K < 1 || R < 1) return kLinearHeader;
@@ -339,21 +396,20 @@ nvfp4_status nvfp4_linear_lora(const void* x, int64_t M, int64_t K, int64_t ld_x
   if (st != NVFP4_OK) return st;
   ++nvfp4::g_last_launches;
   const uint16_t* lb = static_cast<const uint16_t*>(lora_b);
-  if (M <= 32) {
-    st = from_cuda(nvfp4::launch_decode_quantize_x_lora(
-        xb, M, K, ld_x, x_global_scale, x_global_scale ? nullptr : amax_word, w_codes, w_scales, w_global_scale, N,
-        lb, thi, tlo, R, static_cast<uint16_t*>(c), ldc, status, ws + l.gemm_scratch, s));
-    if (st == NVFP4_OK) ++nvfp4::g_last_launches;
-    return st;
-  }
   float* a_gs = x_global_scale ? nullptr : reinterpret_cast<float*>(ws + 260);
   st = from_cuda(nvfp4::launch_quantize(xb, M, K, ld_x, NVFP4_SCALE_ABSMAX, true, x_global_scale, amax_word,
                                         ws + l.x_codes, ws + l.x_scales, a_gs, nullptr, s));
   if (st != NVFP4_OK) return st;
   ++nvfp4::g_last_launches;
-  st = from_cuda(nvfp4::launch_gemm_lora(ws + l.x_codes, ws + l.x_scales, x_global_scale ? x_global_scale : a_gs, M,
-                                         w_codes, w_scales, w_global_scale, N, K, static_cast<uint16_t*>(c), ldc,
-                                         status, lb, thi, tlo, R, s));
+  const float* gs = x_global_scale ? x_global_scale : a_gs;
+  if (M <= 32)
+    st = from_cuda(nvfp4::launch_decode_lora(ws + l.x_codes, ws + l.x_scales, gs, M, w_codes, w_scales,
+                                             w_global_scale, N, K, lb, thi, tlo, R, static_cast<uint16_t*>(c), ldc,
+                                             status, ws + l.gemm_scratch, s));
+  else
+    st = from_cuda(nvfp4::launch_gemm_lora(ws + l.x_codes, ws + l.x_scales, gs, M, w_codes, w_scales,
+                                           w_global_scale, N, K, static_cast<uint16_t*>(c), ldc, status, lb, thi, tlo,
+                                           R, s));
   if (st == NVFP4_OK) ++nvfp4::g_last_launches;
   return st;
 }

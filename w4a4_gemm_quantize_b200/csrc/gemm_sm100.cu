@@ -998,7 +998,42 @@ __global__ void __launch_bounds__(DecodeCfg<QX, LR>::THREADS)
   const int64_t u0 = static_cast<int64_t>(blockIdx.x) * U / G;
   const int64_t u1 = (static_cast<int64_t>(blockIdx.x) + 1) * U / G;
 
-  if (threadIdx.x == 0) {
+  // A unit's loads: its weight part (the 128-row weight tile's K-tile and scale atoms,
+  // plus the stage's byte count for the whole unit) and its activation part.
+  auto issue_weight = [&](int s, int64_t u) {
+    const int tile = static_cast<int>(u / KT), kt = static_cast<int>(u - tile * KT);
+    // scale atoms of the K-tile: four of 64 values (NVFP4) or two of 128 values (MXFP4)
+    constexpr int kAtoms = MX ? 2 : 4;
+    const int sf_atoms = MX ? (K + 127) / 128 : k_atoms;
+    const int ka0 = kt * kAtoms;
+    const uint32_t sf_bytes = static_cast<uint32_t>(min(kAtoms, sf_atoms - ka0)) * Cfg::SF_ATOM;
+    if constexpr (QX) {
+      mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + sf_bytes);
+    } else {
+      mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + 2 * sf_bytes);
+    }
+    tma_load_2d(sA + s * Cfg::A_BYTES, &tmap_w, &full[s], kt * Cfg::KTILE_BYTES, tile * Cfg::BM);
+    bulk_load(sSFA + s * Cfg::SFA_BYTES, sf_w + (static_cast<size_t>(tile) * sf_atoms + ka0) * Cfg::SF_ATOM, sf_bytes,
+              &full[s]);
+  };
+  auto issue_act = [&](int s, int64_t u) {
+    if constexpr (!QX) {
+      const int kt = static_cast<int>(u % KT);
+      constexpr int kAtoms = MX ? 2 : 4;
+      const int sf_atoms = MX ? (K + 127) / 128 : k_atoms;
+      const int ka0 = kt * kAtoms;
+      const uint32_t sf_bytes = static_cast<uint32_t>(min(kAtoms, sf_atoms - ka0)) * Cfg::SF_ATOM;
+      tma_load_2d(sB + s * Cfg::B_BYTES, &tmap_x, &full[s], kt * Cfg::KTILE_BYTES, 0);
+      bulk_load(sSFB + s * Cfg::SFB_BYTES, sf_x + static_cast<size_t>(ka0) * Cfg::SF_ATOM, sf_bytes, &full[s]);
+    }
+  };
+  // The producer thread initialises the barriers and, right away, requests the first
+  // stages' weight parts (the weights do not come from the kernels this one is
+  // launched behind), while the other warps allocate TMEM; the activation parts
+  // follow after the dependency wait.
+  int pre = 0;
+  int64_t pre_u[STAGES];
+  if (warp == 4 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -1014,6 +1049,19 @@ __global__ void __launch_bounds__(DecodeCfg<QX, LR>::THREADS)
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_mbarrier_init();
+    prefetch_tmap(&tmap_w);
+    if (!QX) prefetch_tmap(&tmap_x);
+    if (LR) {
+      prefetch_tmap(&tmap_lb);
+      prefetch_tmap(&tmap_thi);
+      prefetch_tmap(&tmap_tlo);
+    }
+    int64_t s0, s1;
+    for (int sg = 0; pre < STAGES && decode_segment(sg, u0, u1, KT, s0, s1); ++sg)
+      for (int64_t u = s0; u < s1 && pre < STAGES; ++u, ++pre) {
+        issue_weight(pre, u);
+        pre_u[pre] = u;
+      }
   }
   if (QX) {
     // activation rows past M are never written: their codes and scale words stay zero
@@ -1028,19 +1076,11 @@ __global__ void __launch_bounds__(DecodeCfg<QX, LR>::THREADS)
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
-    prefetch_tmap(&tmap_w);
-    if (!QX) prefetch_tmap(&tmap_x);
-    if (LR) {
-      prefetch_tmap(&tmap_lb);
-      prefetch_tmap(&tmap_thi);
-      prefetch_tmap(&tmap_tlo);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+
   // set-up overlapped the previous kernel's tail; its outputs are visible from here
   // (the status word and tile counters were cleared by the memset launched before)
   grid_dependency_wait();
@@ -1050,7 +1090,7 @@ __global__ void __launch_bounds__(DecodeCfg<QX, LR>::THREADS)
       // ---------------- producer ----------------
       int64_t issued_last[STAGES];
 #pragma unroll
-      for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
+      for (int s = 0; s < STAGES; ++s) issued_last[s] = s < pre ? s : -1;
       int64_t i = 0, s0, s1;
       bool ok = true;
       int lora_uses = 0;
@@ -1071,34 +1111,22 @@ __global__ void __launch_bounds__(DecodeCfg<QX, LR>::THREADS)
         }
         for (int64_t u = s0; u < s1; ++u, ++i) {
           const int s = static_cast<int>(i % STAGES);
-          if (!mbar_wait(&empty[s], (static_cast<uint32_t>(i / STAGES) & 1u) ^ 1u, abort_flag, status,
-                         kErrWaitEmpty)) {
-            ok = false;
-            break;
+          if (i >= pre) {  // (units below `pre` have their weight part in flight already)
+            if (!mbar_wait(&empty[s], (static_cast<uint32_t>(i / STAGES) & 1u) ^ 1u, abort_flag, status,
+                           kErrWaitEmpty)) {
+              ok = false;
+              break;
+            }
+            issue_weight(s, u);
           }
-          const int tile = static_cast<int>(u / KT), kt = static_cast<int>(u - tile * KT);
-          // scale atoms of the K-tile: four of 64 values (NVFP4) or two of 128 values (MXFP4)
-          constexpr int kAtoms = MX ? 2 : 4;
-          const int sf_atoms = MX ? (K + 127) / 128 : k_atoms;
-          const int ka0 = kt * kAtoms;
-          const int na = min(kAtoms, sf_atoms - ka0);
-          const uint32_t sf_bytes = static_cast<uint32_t>(na) * Cfg::SF_ATOM;
-          if constexpr (QX) {
-            mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + sf_bytes);
-          } else {
-            mbar_arrive_expect_tx(&full[s], Cfg::A_BYTES + Cfg::B_BYTES + 2 * sf_bytes);
-          }
-          tma_load_2d(sA + s * Cfg::A_BYTES, &tmap_w, &full[s], kt * Cfg::KTILE_BYTES, tile * Cfg::BM);
-          bulk_load(sSFA + s * Cfg::SFA_BYTES, sf_w + (static_cast<size_t>(tile) * sf_atoms + ka0) * Cfg::SF_ATOM,
-                    sf_bytes, &full[s]);
-          if constexpr (!QX) {
-            tma_load_2d(sB + s * Cfg::B_BYTES, &tmap_x, &full[s], kt * Cfg::KTILE_BYTES, 0);
-            bulk_load(sSFB + s * Cfg::SFB_BYTES, sf_x + static_cast<size_t>(ka0) * Cfg::SF_ATOM, sf_bytes, &full[s]);
-          }
+          issue_act(s, u);
           issued_last[s] = i;
         }
       }
       if (*abort_flag) {
+        // a stage whose weight part went out before the wait completes only with its
+        // activation part: send the ones the loop did not reach, then let every copy land
+        for (int64_t j = i; j < pre; ++j) issue_act(static_cast<int>(j), pre_u[j]);
         for (int s = 0; s < STAGES; ++s)
           if (issued_last[s] >= 0)
             mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_last[s] / STAGES) & 1u, status);
@@ -1716,13 +1744,14 @@ size_t gemm_zero_bytes(int64_t M, int64_t N, int64_t) {
 
 cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
-                        uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream) {
+                        uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream, uint8_t* scratch) {
   if (M <= DecodeCfg<false>::BN) {
     CUtensorMap tw, tx;
     if (!encode_codes_map(&tw, b_codes, N, K, 128) || !encode_codes_map(&tx, a_codes, M, K, DecodeCfg<false>::BN))
       return cudaErrorInvalidValue;
+    if (scratch == nullptr) scratch = reinterpret_cast<uint8_t*>(status) + 256;
     return launch_decode<false, false>(tw, tx, tw, tw, tw, 0, a_sf, a_gs, nullptr, 0, nullptr, nullptr, M, b_sf, b_gs,
-                                       N, K, c, ldc, status, reinterpret_cast<uint8_t*>(status) + 256, stream);
+                                       N, K, c, ldc, status, scratch, stream);
   }
   if (M > 128 && N > 128)
     return launch_pair<false, false>(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status, nullptr, nullptr,
@@ -1769,18 +1798,18 @@ cudaError_t launch_gemm_lora(const uint8_t* a_codes, const uint8_t* a_sf, const 
                            stream);
 }
 
-cudaError_t launch_decode_quantize_x_lora(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x,
-                                          const float* x_gs_in, const uint32_t* x_amax, const uint8_t* b_codes,
-                                          const uint8_t* b_sf, const float* b_gs, int64_t N, const uint16_t* lora_b,
-                                          const uint16_t* thi, const uint16_t* tlo, int64_t R, uint16_t* c,
-                                          int64_t ldc, uint32_t* status, uint8_t* scratch, cudaStream_t stream) {
-  CUtensorMap tw, tlb, tth, ttl;
-  if (!encode_codes_map(&tw, b_codes, N, K, 128) || !encode_bf16_rows_map(&tlb, lora_b, N, R, 128) ||
-      !encode_bf16_rows_map(&tth, thi, M, R, DecodeCfg<true, true>::BN) ||
-      !encode_bf16_rows_map(&ttl, tlo, M, R, DecodeCfg<true, true>::BN))
+cudaError_t launch_decode_lora(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
+                               const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
+                               const uint16_t* lora_b, const uint16_t* thi, const uint16_t* tlo, int64_t R,
+                               uint16_t* c, int64_t ldc, uint32_t* status, uint8_t* scratch, cudaStream_t stream) {
+  using Cfg = DecodeCfg<false, true>;
+  CUtensorMap tw, tx, tlb, tth, ttl;
+  if (!encode_codes_map(&tw, b_codes, N, K, 128) || !encode_codes_map(&tx, a_codes, M, K, Cfg::BN) ||
+      !encode_bf16_rows_map(&tlb, lora_b, N, R, 128) || !encode_bf16_rows_map(&tth, thi, M, R, Cfg::BN) ||
+      !encode_bf16_rows_map(&ttl, tlo, M, R, Cfg::BN))
     return cudaErrorInvalidValue;
-  return launch_decode<true, true>(tw, tw, tlb, tth, ttl, static_cast<int>(R), nullptr, nullptr, x, ld_x, x_gs_in,
-                                   x_amax, M, b_sf, b_gs, N, K, c, ldc, status, scratch, stream);
+  return launch_decode<false, true>(tw, tx, tlb, tth, ttl, static_cast<int>(R), a_sf, a_gs, nullptr, 0, nullptr,
+                                    nullptr, M, b_sf, b_gs, N, K, c, ldc, status, scratch, stream);
 }
 
 }  // namespace nvfp4

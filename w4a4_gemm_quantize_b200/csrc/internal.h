@@ -36,10 +36,11 @@ cudaError_t launch_dequantize_mx(const uint8_t* codes, const uint8_t* scales, bo
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t stream);
 
 // GEMM launcher (gemm_sm100.cu).  Returns cudaErrorInvalidValue when a tensor
-// map cannot be encoded.
+// map cannot be encoded.  scratch (M <= 32 only): the small-M kernel's tile counters
+// (zeroed before the launch) and partial tiles; null means status + 256 bytes.
 cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
-                        uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream);
+                        uint16_t* c, int64_t ldc, uint32_t* status, cudaStream_t stream, uint8_t* scratch = nullptr);
 
 // The small-M GEMM (M <= 32) that quantizes its BF16 activation x (M x K, row stride
 // ld_x) itself, absmax block scales under the global scale *x_gs_in, or, when x_gs_in
@@ -50,13 +51,13 @@ cudaError_t launch_decode_quantize_x(const uint16_t* x, int64_t M, int64_t K, in
                                      const float* b_gs, int64_t N, uint16_t* c, int64_t ldc, uint32_t* status,
                                      uint8_t* scratch, cudaStream_t stream);
 
-// The same with the low-rank branch added to the accumulator: lora_b (N x R BF16) and
-// t / alpha as BF16 hi and lo parts (M x R each, from launch_lora_down), R <= 64.
-cudaError_t launch_decode_quantize_x_lora(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x,
-                                          const float* x_gs_in, const uint32_t* x_amax, const uint8_t* b_codes,
-                                          const uint8_t* b_sf, const float* b_gs, int64_t N, const uint16_t* lora_b,
-                                          const uint16_t* thi, const uint16_t* tlo, int64_t R, uint16_t* c,
-                                          int64_t ldc, uint32_t* status, uint8_t* scratch, cudaStream_t stream);
+// The small-M GEMM (M <= 32) on quantized operands with the low-rank branch added to
+// the accumulator: lora_b (N x R BF16) and t / alpha as BF16 hi and lo parts (M x R
+// each, from launch_lora_down), R <= 64; scratch as launch_gemm's.
+cudaError_t launch_decode_lora(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
+                               const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
+                               const uint16_t* lora_b, const uint16_t* thi, const uint16_t* tlo, int64_t R,
+                               uint16_t* c, int64_t ldc, uint32_t* status, uint8_t* scratch, cudaStream_t stream);
 
 // The MXFP4 GEMM C = A B^T (E8M0 block-32 scales, swizzled, no per-tensor scales):
 // the small-M kernel for M <= 32 (workspace as nvfp4_gemm's), the CTA-pair kernel above.

@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(LoraCfg::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  grid_dependency_wait();  // x and the activation's amax word come from earlier kernels
+  grid_dependents_launch();  // the quantizer and GEMM behind this kernel may set up meanwhile
+  grid_dependency_wait();    // x and the activation's amax word come from earlier kernels
 
   if (warp == 0) {
     if (lane == 0) {

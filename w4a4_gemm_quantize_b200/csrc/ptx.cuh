@@ -97,6 +97,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // does before this call must not read what those grids write.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Let the grid launched behind this one (with programmatic dependent launch) start
+// now: it sets up and begins whatever does not depend on this grid's output (it
+// reads that output only after its own grid_dependency_wait, which still waits for
+// this grid to complete).  Every kernel of the library waits before reading.
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ---------------------------------------------------------------------------------------------
 // TMA / bulk copies (global -> shared, completion counted on an mbarrier)
 // ---------------------------------------------------------------------------------------------

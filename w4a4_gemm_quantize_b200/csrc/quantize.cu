@@ -65,6 +65,7 @@ __device__ __forceinline__ uint32_t vmax_mag(uint32_t m, uint4 v) {
 __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                         int64_t cols, int64_t ld,
                                                         uint32_t* __restrict__ amax_bits) {
+  grid_dependents_launch();  // the quantizer behind this pass may set up meanwhile
   uint32_t m = 0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -140,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
     const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ gs_out, float* __restrict__ block_err) {
   __shared__ ScaleTables tab;
-  grid_dependency_wait();  // launched behind the amax pass (programmatic launch)
+  grid_dependents_launch();  // the GEMM behind this pass may set up and start its weight stream
+  grid_dependency_wait();    // launched behind the amax pass (programmatic launch)
   const int64_t nblk = cols / 16;
   const int64_t atoms_per_group = (nblk + 3) / 4;
   const float sg = global_scale(gs_in, amax_bits);
