@@ -90,7 +90,33 @@ def parse_args(argv=None):
 
 
 KERNEL_SOURCES = {"gemm": ["gemm_sm100.cu", "ptx.cuh", "internal.h"],
-                  "quantize": ["quantize.cu", "ptx.cuh", "internal.h"]}
+                  "quantize": ["quantize.cu", "quant_block.cuh", "ptx.cuh", "internal.h"],
+                  "lora": ["lora.cu", "gemm_sm100.cu", "quant_block.cuh", "ptx.cuh", "internal.h"]}
+KERNEL_FAMILY = {"gemm_pair_kernel": "gemm", "gemm_decode_kernel": "gemm", "gemm_kernel": "gemm",
+                 "gemm_pair_kernel_lora": "lora", "gemm_decode_kernel_lora": "lora", "quantize_kernel": "quantize",
+                 "dequantize_kernel": "quantize"}
+
+
+def group_kernel(group: str, cfg: dict, family: str):
+    """(file tag, description) of the kernel that dominates a group's time."""
+    if family == "gemm":
+        n_of = {"gemm_1": "N1", "gemm_2": "N2", "gemm_up": "N_up", "gemm_down": "N_down", "gemm": "N", "linear": "N",
+                "linear_lora": "N", "linear_lora_up": "N_up", "linear_lora_down": "N_down"}
+        M, N = cfg["M"], cfg[n_of[group]]
+        tag = "gemm_decode_kernel" if M <= 32 else ("gemm_pair_kernel" if M > 128 and N > 128 else "gemm_kernel")
+        desc = {"gemm_decode_kernel": "gemm_decode_kernel (tcgen05 mxf4nvf4, 128-row weight tiles)",
+                "gemm_pair_kernel": "gemm_pair_kernel (tcgen05 cta_group::2 mxf4nvf4)",
+                "gemm_kernel": "gemm_kernel (tcgen05 mxf4nvf4)"}[tag]
+        if group == "linear":
+            desc = "quantize_kernel + " + desc + " (one nvfp4_linear call)"
+        if group.startswith("linear_lora"):
+            tag += "_lora"
+            desc = ("lora_down_kernel + quantize_kernel + " + desc +
+                    " with the low-rank MMAs in the FP4 accumulator (one nvfp4_linear_lora call)")
+        return tag, desc
+    if group.startswith("quantize"):
+        return "quantize_kernel", "amax_kernel + quantize_kernel"
+    return "dequantize_kernel", "dequantize_kernel"
 
 
 def source_hash(kernel: str = "gemm") -> str:
@@ -114,10 +140,11 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sust=1400.0, source="fallback")
 
 
-def profiled_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, only if it was taken on
-    the current kernel sources (the summary records the source hash)."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+def profiled_traffic(tag: str, workload: str, group: str):
+    """DRAM bytes per launch of a group's dominant kernel from the committed ncu summary
+    profiles/<kernel>_<workload>_<group>.md, only if it was taken on the current kernel
+    sources (the summary records their hash)."""
+    path = os.path.join(ROOT, "profiles", f"{tag}_{workload}_{group}.md")
     if not os.path.exists(path):
         return None
     vals = {}
@@ -126,7 +153,7 @@ def profiled_traffic(kernel: str, workload: str):
             if ":" in line and line.startswith("- "):
                 k, v = line[2:].split(":", 1)
                 vals[k.strip()] = v.strip().strip("`")
-    if vals.get("source_hash") != source_hash(kernel):
+    if vals.get("source_hash") != source_hash(KERNEL_FAMILY[tag]):
         return None
     try:
         return float(vals["traffic_bytes_per_launch"])
@@ -253,15 +280,6 @@ def lora_work(M, N, K, R):
     w = gemm_work(M, N, K)
     return {"flops": w["flops"] + 2.0 * M * K * R + 2.0 * M * N * R,
             "bytes": N * K * 0.5625 + M * K * 2.0 + (R * K + N * R) * 2.0 + 2.0 * M * N}
-
-
-def gemm_kernel_name(M: int, N: int) -> str:
-    """The kernel the library picks for an M x N output (its launch dispatch)."""
-    if M <= 32:
-        return "gemm_decode_kernel (tcgen05 mxf4nvf4, stream-K)"
-    if M > 128 and N > 128:
-        return "gemm_pair_kernel (tcgen05 cta_group::2 mxf4nvf4)"
-    return "gemm_kernel (tcgen05 mxf4nvf4)"
 
 
 def host_inputs(cfg, seed: int, rank: int):
@@ -611,18 +629,8 @@ def run_ours(args, rank, world, local, host):
         comps[n] = {"us": round(per_group[n], 2), r["unit"]: r["achieved"], "frac": r["frac"], "bound": r["bound"]}
     dom = max(names, key=lambda n: per_group[n])
     roof = group_rate(works[dom], per_group[dom], peaks, long_region)
-    if families[dom] == "gemm":
-        n_of = {"gemm_1": "N1", "gemm_2": "N2", "gemm_up": "N_up", "gemm_down": "N_down", "gemm": "N", "linear": "N",
-                "linear_lora": "N", "linear_lora_up": "N_up", "linear_lora_down": "N_down"}
-        kname = gemm_kernel_name(cfg["M"], cfg[n_of[dom]])
-        if dom == "linear":
-            kname = "gemm_decode_kernel<true> (activation quantized in the GEMM; tcgen05 mxf4nvf4, stream-K)"
-        if dom.startswith("linear_lora"):
-            kname = ("lora_down_kernel + " + ("gemm_decode_kernel<true, true>" if cfg["M"] <= 32 else
-                     "quantize_kernel + gemm_pair_kernel<true>") + " (low-rank MMAs in the FP4 accumulator)")
-    else:
-        kname = "amax_kernel + quantize_kernel" if dom.startswith("quantize") else "dequantize_kernel"
-    roof.update({"traffic": profiled_traffic(families[dom], f"{dom}_{args.workload}"),
+    tag, kname = group_kernel(dom, cfg, families[dom])
+    roof.update({"traffic": profiled_traffic(tag, args.workload, dom),
                  "kernel": f"{kname}, group {dom}", "group_share_of_step": round(per_group[dom] / (step_ms * 1e3), 4)})
     roof = {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "kernel", "peak_source",
                                  "group_share_of_step")}

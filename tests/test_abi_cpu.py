@@ -166,11 +166,14 @@ def test_bench_profile_record_matches_only_its_sources(tmp_path, monkeypatch):
     os.symlink(real_csrc, tmp_path / "w4a4_gemm_quantize_b200" / "csrc")
     os.makedirs(tmp_path / "profiles")
     h = bench.source_hash("gemm")
-    (tmp_path / "profiles" / "gemm_w.md").write_text(f"- source_hash: `{h}`\n- traffic_bytes_per_launch: 1234\n")
-    assert bench.profiled_traffic("gemm", "w") == 1234.0
-    (tmp_path / "profiles" / "gemm_w.md").write_text("- source_hash: `0000000000000000`\n- traffic_bytes_per_launch: 1234\n")
-    assert bench.profiled_traffic("gemm", "w") is None
-    assert bench.profiled_traffic("gemm", "missing") is None
+    f = tmp_path / "profiles" / "gemm_pair_kernel_w_gemm_1.md"
+    f.write_text(f"- source_hash: `{h}`\n- traffic_bytes_per_launch: 1234\n")
+    assert bench.profiled_traffic("gemm_pair_kernel", "w", "gemm_1") == 1234.0
+    f.write_text("- source_hash: `0000000000000000`\n- traffic_bytes_per_launch: 1234\n")
+    assert bench.profiled_traffic("gemm_pair_kernel", "w", "gemm_1") is None
+    assert bench.profiled_traffic("gemm_pair_kernel", "missing", "gemm_1") is None
+    # a low-rank group's kernel is hashed with the down-projection's sources too
+    assert bench.KERNEL_FAMILY["gemm_pair_kernel_lora"] == "lora" and "lora.cu" in bench.KERNEL_SOURCES["lora"]
 
 
 def test_noalloc_validation_before_any_cuda_call(lib):

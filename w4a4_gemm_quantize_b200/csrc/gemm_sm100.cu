@@ -357,13 +357,15 @@ struct PairCfg {
   static constexpr int SFA_BYTES = 4 * SF_ATOM;       // own 128 rows, 4 K-steps
   static constexpr int SFB_BYTES = 2 * 4 * SF_ATOM;   // all 256 rows, 4 K-steps
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  // LR (low-rank branch): four stages, C written with direct stores (no staging boxes),
-  // and the tile's low-rank operands -- t / alpha hi and lo (this CTA's 128 rows) and
-  // B's rows (this CTA's 128 columns), 128-byte K-major rows (rank up to 64)
+  // LR (low-rank branch): four stages, C staged through 32 x 32 boxes (64-byte swizzle)
+  // instead of 32 x 64, and the tile's low-rank operands -- t / alpha hi and lo (this
+  // CTA's 128 rows) and B's rows (this CTA's 128 columns), 128-byte K-major rows
+  // (rank up to 64)
   static constexpr int STAGES = LR ? 4 : 5;
   static constexpr int EPI_WARPS = 8;
-  static constexpr int C_BOX_BYTES = 32 * 128;        // 32 rows x 64 BF16 columns
-  static constexpr int C_BYTES = LR ? 0 : EPI_WARPS * C_BOX_BYTES;
+  static constexpr int C_BOX_COLS = LR ? 32 : 64;     // BF16 columns of one staging box
+  static constexpr int C_BOX_BYTES = 32 * C_BOX_COLS * 2;
+  static constexpr int C_BYTES = EPI_WARPS * C_BOX_BYTES;
   static constexpr int LORA_BYTES = LR ? 3 * 128 * 128 : 0;
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + C_BYTES + LORA_BYTES + BAR_BYTES;
@@ -453,12 +455,11 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
     prefetch_tmap(&tmap_b);
     prefetch_tmap(&tmap_sfa);
     prefetch_tmap(&tmap_sfb);
+    prefetch_tmap(&tmap_c);
     if (LR) {
       prefetch_tmap(&tmap_lb);
       prefetch_tmap(&tmap_thi);
       prefetch_tmap(&tmap_tlo);
-    } else {
-      prefetch_tmap(&tmap_c);
     }
   }
   tc_fence_before();
@@ -770,18 +771,27 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
       const int row0 = tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM + quarter * 32;
       const int col0 = tn * Cfg::BN + half * HALF;
       if constexpr (LR) {
-        // row row0 + lane, columns [col0, col0 + 128): 16-byte stores from registers
-        const int row = row0 + lane;
-        if (row < M && col0 < N) {
-          uint16_t* dst = C + static_cast<int64_t>(row) * ldc + col0;
-          if (col0 + HALF <= N) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
+        // four 32 x 32 boxes per warp, 64-byte swizzle: 16-byte unit u of row `lane` goes to
+        // u ^ ((lane / 2) % 4)
 #pragma unroll
-            for (int i = 0; i < HALF / 8; ++i) d4[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-          } else {
-            for (int i = 0; i < HALF; ++i)
-              if (col0 + i < N) dst[i] = static_cast<uint16_t>((i & 1) ? (p[i >> 1] >> 16) : (p[i >> 1] & 0xFFFFu));
+        for (int chunk = 0; chunk < 4; ++chunk) {
+          if (stored) {  // the previous TMA store from this box must have read it
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
           }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int q = chunk * 16 + 4 * u;
+            *reinterpret_cast<uint4*>(box + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(p[q], p[q + 1], p[q + 2], p[q + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < M && col0 + chunk * 32 < N) {
+            tma_store_2d(&tmap_c, box, col0 + chunk * 32, row0);
+            bulk_commit_group();
+          }
+          stored = true;
         }
       } else {
 #pragma unroll
@@ -1571,16 +1581,18 @@ int max_pair_clusters(int dev) {
 }
 
 // BF16 output matrix, row stride ldc elements; box = 32 rows x 64 columns, 128-byte swizzle.
-bool encode_c_map(CUtensorMap* map, uint16_t* c, int64_t M, int64_t N, int64_t ldc) {
+// BF16 M x N output (row stride ldc), box = 32 rows x box_cols (64: 128-byte swizzle,
+// 32: 64-byte swizzle).
+bool encode_c_map(CUtensorMap* map, uint16_t* c, int64_t M, int64_t N, int64_t ldc, int box_cols = 64) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldc * 2)};
-  const cuuint32_t box[2] = {64u, 32u};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), 32u};
   const cuuint32_t estr[2] = {1u, 1u};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // BF16 rows x R matrix (row stride R elements, R <= 64): box = box_rows x 64 values
@@ -1607,7 +1619,7 @@ cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float
   CUtensorMap ta, tb, tsa, tsb, tc, tlb, tth, ttl;
   if (!encode_codes_map(&ta, a_codes, M, K, 128) || !encode_codes_map(&tb, b_codes, N, K, 128) ||
       !encode_sf_map(&tsa, a_sf, M, K, 1, MX) || !encode_sf_map(&tsb, b_sf, N, K, 2, MX) ||
-      !encode_c_map(&tc, c, M, N, ldc))
+      !encode_c_map(&tc, c, M, N, ldc, Cfg::C_BOX_COLS))
     return cudaErrorInvalidValue;
   if (LR) {
     if (!encode_bf16_rows_map(&tlb, lora_b, N, rank, 128) || !encode_bf16_rows_map(&tth, thi, M, rank, 128) ||

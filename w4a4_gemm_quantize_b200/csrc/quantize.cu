@@ -172,16 +172,43 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
     c_step = nwarps;
   }
   const int lane = threadIdx.x & 31;
-  for (int64_t r = r0; r < rows; r += r_step) {
+  // absmax and four-over-six: the warp's next 32 blocks are requested before these are
+  // encoded, so two blocks' loads per lane are in flight (the MSE search is issue-bound
+  // and keeps its registers)
+  constexpr bool kPrefetch = MODE != 1;
+  auto load_block = [&](int64_t r, int64_t c, uint4& lo, uint4& hi) {
+    const int64_t cb = c * 32 + lane;
+    if (r < rows && cb < nblk) {
+      const uint16_t* p = x + r * ld + cb * 16;
+      lo = ld_nc_v4(p);
+      hi = ld_nc_v4(p + 8);
+    }
+  };
+  uint4 next_lo = make_uint4(0u, 0u, 0u, 0u), next_hi = next_lo;
+  if (c0 >= chunks) r0 = rows;
+  if (kPrefetch) load_block(r0, c0, next_lo, next_hi);
+  // (r, c) walks the warp's tasks in order: c = c0, c0 + c_step, ... below `chunks` for
+  // r = r0, r0 + r_step, ...
+  for (int64_t r = r0, c = c0; r < rows;) {
+    int64_t rn = r, cn = c + c_step;
+    if (cn >= chunks) {
+      cn = c0;
+      rn = r + r_step;
+    }
+    uint4 lo = next_lo, hi = next_hi;
+    if (kPrefetch) load_block(rn, cn, next_lo, next_hi);
     const uint16_t* xrow = x + r * ld;
     uint8_t* crow = codes + r * (cols / 2);
     const int64_t sf_row = SWZ ? (r >> 7) * atoms_per_group * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 : r * nblk;
-    for (int64_t c = c0; c < chunks; c += c_step) {
+    {
       const int64_t cb = c * 32 + lane;
       const bool active = cb < nblk;
       uint32_t best_s = 0;
       if (active) {
-        const uint4 lo = ld_nc_v4(xrow + cb * 16), hi = ld_nc_v4(xrow + cb * 16 + 8);
+        if (!kPrefetch) {
+          lo = ld_nc_v4(xrow + cb * 16);
+          hi = ld_nc_v4(xrow + cb * 16 + 8);
+        }
         const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
         uint64_t x2[8];  // the block as signed binary32 pairs (BF16 widening is exact)
         uint32_t mb = 0;
@@ -265,6 +292,8 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
               best_s | (s1 << 8) | (s2 << 16) | (s3 << 24);
       }
     }
+    r = rn;
+    c = cn;
   }
   if (SWZ) zero_scale_padding(scales, rows, nblk);
 }
