@@ -132,6 +132,70 @@ __device__ __forceinline__ void zero_scale_padding(uint8_t* __restrict__ scales,
   }
 }
 
+// Load one 16-value block: its binary32 pairs, its maximum magnitude and
+// v_b = amax_b / (6 s_g).
+__device__ __forceinline__ void load_x2(uint4 lo, uint4 hi, float d6, uint64_t (&x2)[8], float& amax_b,
+                                        float& vb) {
+  const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  uint32_t mb = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x2[i] = pack2(__uint_as_float(wd[i] << 16), __uint_as_float(wd[i] & 0xFFFF0000u));  // exact widening
+    mb = __vmaxu2(mb, wd[i] & 0x7FFF7FFFu);
+  }
+  amax_b = bf16_bits_to_float(max(mb & 0xFFFFu, mb >> 16));
+  vb = __fdiv_rn(amax_b, d6);
+}
+
+// Clip bound of the MSE walk: if the block maximum lands above the 4|6 midpoint it
+// is coded as 6, and its term alone makes e >= RN(d*d) with d = fma(-6, eff, amax_b):
+// each fma of the error sum adds a non-negative term to a non-negative sum, and
+// rounding is monotone.  Such a candidate cannot strictly improve when RN(d*d) >=
+// best_e.  When d >= 0 (the maximum is clipped) later candidates, with smaller eff,
+// have a larger d and cannot either, so the walk stops.
+enum Verdict { kEvaluate, kSkip, kStop };
+__device__ __forceinline__ Verdict clip_verdict(float amax_b, float eff, float rcp, float best_e) {
+  if (eff != 0.0f && __fmul_rn(amax_b, rcp) > 5.0f) {
+    const float d = __fmaf_rn(-6.0f, eff, amax_b);
+    if (__fmul_rn(d, d) >= best_e) return d >= 0.0f ? kStop : kSkip;
+  }
+  return kEvaluate;
+}
+
+// Evaluate scale s in full and keep it on a strict improvement.
+__device__ __forceinline__ void mse_try(const uint64_t (&x2)[8], uint32_t s, float eff, float rcp, uint32_t& best_s,
+                                        float& best_e, uint32_t& best_c0, uint32_t& best_c1) {
+  uint32_t c0w, c1w;
+  encode_codes(x2, eff, rcp, c0w, c1w);
+  const float e = block_sse(x2, c0w, c1w, eff);
+  if (e < best_e) {
+    best_e = e;
+    best_s = s;
+    best_c0 = c0w;
+    best_c1 = c1w;
+  }
+}
+
+// The MSE walk over the candidates f = 0.9, 0.8, ..., 0.3 (index i = 0..6) from
+// index i0, with prev_s the scale of the candidate before it.
+__device__ __forceinline__ void mse_walk(const uint64_t (&x2)[8], float amax_b, float vb, int i0, uint32_t prev_s,
+                                         const ScaleTables& tab, uint32_t& best_s, float& best_e, uint32_t& best_c0,
+                                         uint32_t& best_c1) {
+#pragma unroll 1
+  for (int i = i0; i < 7; ++i) {
+    // the factor of candidate i, selected in registers (an indexed array would live in
+    // local memory)
+    const float fi = i == 0 ? 0.9f : i == 1 ? 0.8f : i == 2 ? 0.7f : i == 3 ? 0.6f : i == 4 ? 0.5f : i == 5 ? 0.4f : 0.3f;
+    const uint32_t s = cvt_e4m3_satfinite(__fmul_rn(fi, vb));
+    if (s == prev_s) continue;  // same scale, same error: never a strict improvement
+    prev_s = s;
+    const float eff = tab.eff[s], rcp = tab.rcp[s];
+    const Verdict v = clip_verdict(amax_b, eff, rcp, best_e);
+    if (v == kStop) return;
+    if (v == kEvaluate) mse_try(x2, s, eff, rcp, best_s, best_e, best_c0, best_c1);
+  }
+}
+
 // One warp handles 32 consecutive blocks of one row (lane = block); warps walk a
 // fixed column chunk down the rows, so block coordinates and output offsets need
 // no division.
@@ -141,6 +205,15 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
     const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ gs_out, float* __restrict__ block_err) {
   __shared__ ScaleTables tab;
+  // MSE: per-warp ring of blocks whose walk goes on past f = 0.9 (about one block in
+  // seven, but nearly every warp has one).  They are resumed 32 at a time, one per
+  // lane, so the longer walks no longer hold the other 31 lanes of a warp.  An entry
+  // is three 16-byte words: {row r, block column cb, the scales (current best, last
+  // candidate) with bits 32..39 of cb and of r, error}, then the block's 16 BF16 values
+  // (a tensor in device memory has fewer than 2^40 rows and blocks per row).  A resumed block that
+  // finds no better scale keeps the outputs already stored, so its codes are not kept.
+  constexpr int kRing = MODE == 1 ? 64 : 1;
+  __shared__ uint4 ring[3][kThreads / 32][kRing];
   grid_dependents_launch();  // the GEMM behind this pass may set up and start its weight stream
   grid_dependency_wait();    // launched behind the amax pass (programmatic launch)
   const int64_t nblk = cols / 16;
@@ -172,6 +245,32 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
     c_step = nwarps;
   }
   const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  uint32_t ring_head = 0, ring_tail = 0;  // warp-uniform
+  // resume the walks of the n oldest queued blocks (lane j takes the j-th) and rewrite
+  // the outputs of those whose best candidate changed
+  auto resume = [&](uint32_t n) {
+    __syncwarp();
+    const uint32_t slot = (ring_head + lane) & (kRing - 1);
+    const uint4 f = ring[0][wid][slot], lo = ring[1][wid][slot], hi = ring[2][wid][slot];
+    __syncwarp();  // the slots may be refilled once every lane has read its entry
+    ring_head += n;
+    if (static_cast<uint32_t>(lane) >= n) return;
+    const int64_t r = static_cast<int64_t>((static_cast<uint64_t>(f.z >> 24) << 32) | f.x);
+    const int64_t cb = static_cast<int64_t>((static_cast<uint64_t>((f.z >> 16) & 0xFFu) << 32) | f.y);
+    uint64_t x2[8];
+    float amax_b, vb;
+    load_x2(lo, hi, d6, x2, amax_b, vb);
+    uint32_t best_s = f.z & 0xFFu;
+    const uint32_t queued_s = best_s;
+    float best_e = __uint_as_float(f.w);
+    uint32_t best_c0 = 0, best_c1 = 0;
+    mse_walk(x2, amax_b, vb, 1, (f.z >> 8) & 0xFFu, tab, best_s, best_e, best_c0, best_c1);
+    if (best_s == queued_s) return;  // a strict improvement always changes the scale
+    *reinterpret_cast<uint2*>(codes + r * (cols / 2) + cb * 8) = make_uint2(best_c0, best_c1);
+    scales[SWZ ? swizzled_offset(r, cb, atoms_per_group) : r * nblk + cb] = static_cast<uint8_t>(best_s);
+    if (block_err) block_err[r * nblk + cb] = best_e;
+  };
   // absmax and four-over-six: the warp's next 32 blocks are requested before these are
   // encoded, so two blocks' loads per lane are in flight (the MSE search is issue-bound
   // and keeps its registers)
@@ -204,21 +303,16 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
       const int64_t cb = c * 32 + lane;
       const bool active = cb < nblk;
       uint32_t best_s = 0;
+      uint32_t n_queued = 0;  // MSE: blocks of this task queued (valid in lane 0)
+      const uint32_t active_mask = MODE == 1 ? __ballot_sync(0xFFFFFFFFu, active) : 0u;
       if (active) {
         if (!kPrefetch) {
           lo = ld_nc_v4(xrow + cb * 16);
           hi = ld_nc_v4(xrow + cb * 16 + 8);
         }
-        const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        uint64_t x2[8];  // the block as signed binary32 pairs (BF16 widening is exact)
-        uint32_t mb = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          x2[i] = pack2(__uint_as_float(wd[i] << 16), __uint_as_float(wd[i] & 0xFFFF0000u));
-          mb = __vmaxu2(mb, wd[i] & 0x7FFF7FFFu);
-        }
-        const float amax_b = bf16_bits_to_float(max(mb & 0xFFFFu, mb >> 16));
-        const float vb = __fdiv_rn(amax_b, d6);
+        uint64_t x2[8];  // the block as signed binary32 pairs
+        float amax_b, vb;
+        load_x2(lo, hi, d6, x2, amax_b, vb);
 
         // candidate f = 1: the absmax scale
         best_s = cvt_e4m3_satfinite(vb);
@@ -229,37 +323,40 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
         if (MODE != 0 || block_err) best_e = block_sse(x2, best_c0, best_c1, best_eff);
 
         if (MODE == 1) {
-          const float factors[7] = {0.9f, 0.8f, 0.7f, 0.6f, 0.5f, 0.4f, 0.3f};
+          // f = 0.9 here, and the clip test of f = 0.8; a block whose walk goes on is
+          // queued with its state and resumes at f = 0.8
           uint32_t prev_s = best_s;
-#pragma unroll 1
-          for (int i = 0; i < 7; ++i) {
-            const uint32_t s = cvt_e4m3_satfinite(__fmul_rn(factors[i], vb));
-            if (s == prev_s) continue;  // same scale, same error: never a strict improvement
+          bool more = true;
+          uint32_t s = cvt_e4m3_satfinite(__fmul_rn(0.9f, vb));
+          if (s != prev_s) {
             prev_s = s;
             const float eff = tab.eff[s], rcp = tab.rcp[s];
-            // Clip bound: if the block maximum lands above the 4|6 midpoint it is coded
-            // as 6, and its term alone makes e >= RN(d*d) with d = fma(-6, eff, amax_b):
-            // each fma of the error sum adds a non-negative term to a non-negative sum,
-            // and rounding is monotone.  Such a candidate cannot strictly improve when
-            // RN(d*d) >= best_e.  When d >= 0 (the maximum is clipped) later candidates,
-            // with smaller eff, have a larger d and cannot either, so the walk stops.
-            if (eff != 0.0f && __fmul_rn(amax_b, rcp) > 5.0f) {
-              const float d = __fmaf_rn(-6.0f, eff, amax_b);
-              if (__fmul_rn(d, d) >= best_e) {
-                if (d >= 0.0f) break;
-                continue;
-              }
-            }
-            uint32_t c0w, c1w;
-            encode_codes(x2, eff, rcp, c0w, c1w);
-            const float e = block_sse(x2, c0w, c1w, eff);
-            if (e < best_e) {
-              best_e = e;
-              best_s = s;
-              best_c0 = c0w;
-              best_c1 = c1w;
-            }
+            const Verdict v = clip_verdict(amax_b, eff, rcp, best_e);
+            more = v != kStop;
+            if (v == kEvaluate) mse_try(x2, s, eff, rcp, best_s, best_e, best_c0, best_c1);
           }
+          if (more) {
+            s = cvt_e4m3_satfinite(__fmul_rn(0.8f, vb));
+            if (s != prev_s) more = clip_verdict(amax_b, tab.eff[s], tab.rcp[s], best_e) != kStop;
+          }
+          // the outputs below hold the best so far; a queued block's are rewritten when
+          // it is resumed (active lanes are a prefix of the warp, lane 0 among them)
+          const uint32_t queued = __ballot_sync(active_mask, more);
+          if (more) {
+            const uint32_t slot = (ring_tail + __popc(queued & ((1u << lane) - 1u))) & (kRing - 1);
+            const uint32_t hi_bits = ((static_cast<uint32_t>(static_cast<uint64_t>(cb) >> 32) & 0xFFu) << 16) |
+                                     (static_cast<uint32_t>(static_cast<uint64_t>(r) >> 32) << 24);
+            ring[0][wid][slot] = make_uint4(static_cast<uint32_t>(r), static_cast<uint32_t>(cb),
+                                            best_s | (prev_s << 8) | hi_bits, __float_as_uint(best_e));
+            // each BF16 pair back from its exact binary32 widening: the high halves
+            uint32_t wd[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              wd[j] = __byte_perm(static_cast<uint32_t>(x2[j]), static_cast<uint32_t>(x2[j] >> 32), 0x7632);
+            ring[1][wid][slot] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            ring[2][wid][slot] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+          }
+          n_queued = __popc(queued);
         }
         if (MODE == 2) {
           // four-over-six: the block maximum mapped to 4 instead of 6, kept only on a
@@ -291,10 +388,15 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
           *reinterpret_cast<uint32_t*>(scales + sf_row + (cb >> 2) * 512) =
               best_s | (s1 << 8) | (s2 << 16) | (s3 << 24);
       }
+      if (MODE == 1) {
+        ring_tail += __shfl_sync(0xFFFFFFFFu, n_queued, 0);
+        if (ring_tail - ring_head >= 32) resume(32);  // at most 63 queued before this
+      }
     }
     r = rn;
     c = cn;
   }
+  if (MODE == 1 && ring_tail != ring_head) resume(ring_tail - ring_head);
   if (SWZ) zero_scale_padding(scales, rows, nblk);
 }
 
