@@ -123,11 +123,17 @@ nvfp4_status nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, nvfp4
                               int64_t ld_out, void *stream);
 
 /* Workspace nvfp4_gemm needs (device memory, any content on entry): 256 bytes
- * for the status word, plus, when M <= 32, the small-M kernel's per-tile counters
- * and FP32 partial tiles (the weight stream is split evenly over the SMs, so a
- * 128-row weight tile can be cut into a few K segments: about
- * N * 128 * segments bytes, a few MB for 8B-class layers).  nvfp4_gemm clears the
- * status word and the counters itself (one memset on `stream`). */
+ * for the status word, plus
+ *  - when M <= 32, the small-M kernel's per-tile counters and FP32 partial tiles
+ *    (the weight stream is split evenly over the SMs, so a 128-row weight tile can
+ *    be cut into a few K segments: about N * 128 * segments bytes, a few MB for
+ *    8B-class layers);
+ *  - when M > 128 and N > 128, the 256 x 256-tile kernel's shared-tile counters and
+ *    FP32 partial tiles (when the tile count is not a multiple of the CTA pairs and
+ *    K is long, the last round's work is spread over all pairs, a tile split along K
+ *    between two of them; 74 slots of 512 KB, about 38.8 MB).
+ * nvfp4_gemm clears the status word and the counters itself (one memset on
+ * `stream`). */
 size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Block-scaled W4A4 GEMM, C = (A s_a)(B s_b)^T * s_gA * s_gB, FP32 accumulation,

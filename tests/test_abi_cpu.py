@@ -118,9 +118,15 @@ def test_decode_workspace_holds_every_partial_tile():
         segs = min(KT, (KT - 1) // per + 2)
         counters = -(-(T * 4) // 256) * 256
         assert lib.nvfp4_gemm_workspace_bytes(M, N, K) == 256 + counters + T * segs * 128 * 32 * 4, (M, N, K)
-    # larger M needs only the status block
+    # M in 33..128 (or N <= 128): only the status block
     assert lib.nvfp4_gemm_workspace_bytes(33, 14336, 4096) == 256
-    assert lib.nvfp4_gemm_workspace_bytes(8192, 21504, 5376) == 256
+    assert lib.nvfp4_gemm_workspace_bytes(4096, 128, 4096) == 256
+    # M, N > 128 (CTA pairs on 256 x 256 tiles): a ticket and a flag word per slot, CTA and
+    # epilogue warp for 74 slots (rounded up to 256 bytes), then per slot two pieces x two
+    # CTAs x 8 warps x 32 x 128 FP32 partial sums
+    pair = 256 + -(-(2 * 74 * 2 * 8 * 4) // 256) * 256 + 74 * 2 * 2 * 8 * 32 * 128 * 4
+    for (M, N, K) in [(8192, 21504, 5376), (129, 129, 32), (256, 5376, 21504)]:
+        assert lib.nvfp4_gemm_workspace_bytes(M, N, K) == pair, (M, N, K)
 
 
 def test_dequantize_validation(lib):

@@ -147,6 +147,26 @@ def test_prefill_down_projection_sampled(cuda_device):
     _sampled(M, N, K, a, b, out, seed=1)
 
 
+def test_shared_tiles_stream_k_sampled(cuda_device):
+    """M=2560, N=2048, K=12288: 80 tiles of 256 x 256 on the CTA pairs with 48 K-tiles
+    each, so the last round's work is spread over every pair and most tiles are split
+    along K between two pairs (partial sums through the workspace, the second piece adds
+    them).  Sampled outputs against the FP64 reference, two launches bitwise equal on a
+    workspace whose content on entry is arbitrary, no device-side timeout."""
+    M, N, K = 2560, 2048, 12288
+    a = oracle_operand(workloads.activation(M, K, seed=5, n_outlier_channels=4))
+    b = oracle_operand(workloads.gaussian_weight(N, K, 0.02, seed=5), oracle.SCALE_MSE)
+    A, B = upload(a), upload(b)
+    ws_bytes = nv.load_library().nvfp4_gemm_workspace_bytes(M, N, K)
+    ws = torch.full((ws_bytes,), 0xAB, dtype=torch.uint8, device="cuda")
+    out = nv.nvfp4_gemm(A, B, workspace=ws)
+    assert nv.read_device_error(ws) == 0
+    out2 = nv.nvfp4_gemm(A, B, workspace=ws)
+    assert nv.read_device_error(ws) == 0
+    assert torch.equal(out, out2)
+    _sampled(M, N, K, a, b, out, n_samples=8000, seed=5)
+
+
 def test_scaled_mm_library_pin_of_the_oracle(cuda_device):
     """Pin the oracle's nibble order and swizzled scale layout against a library
     routine: torch._scaled_mm (cuBLASLt NVFP4) reads the oracle's bytes and must

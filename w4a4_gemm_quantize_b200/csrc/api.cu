@@ -38,8 +38,8 @@ nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVF
 
 // Workspace of nvfp4_linear: [0, 256) the GEMM status word, [256, 260) the
 // activation's amax word, [260, 264) its global scale (large-M path), then from
-// byte 512 either the small-M kernel's counters and partial tiles or the
-// activation's codes (rounded up to 256 bytes) and swizzled scales.
+// byte 512 the GEMM's counters and partial tiles (small-M kernel or pair kernel),
+// and the activation's codes (rounded up to 256 bytes) and swizzled scales.
 constexpr size_t kLinearHeader = 512;
 
 size_t linear_codes_bytes(int64_t M, int64_t K) { return (static_cast<size_t>(M) * (K / 2) + 255) / 256 * 256; }
@@ -210,9 +210,9 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const f
 namespace {
 
 // Workspace of nvfp4_linear: the 512-byte header (status word, amax word, the
-// activation's global scale), for M <= 32 the small-M GEMM's counters and partial
-// tiles, then the activation's codes and swizzled scales.  The memset clears the
-// header and the counters (the `zero` bytes).
+// activation's global scale), the GEMM's counters and partial tiles, then the
+// activation's codes and swizzled scales.  The memset clears the header and the
+// counters (the `zero` bytes).
 struct LinearLayout {
   size_t gemm_scratch, x_codes, x_scales, zero, total;
 };
@@ -220,8 +220,8 @@ struct LinearLayout {
 LinearLayout linear_layout(int64_t M, int64_t N, int64_t K) {
   LinearLayout l{};
   l.gemm_scratch = kLinearHeader;
-  const size_t scratch = M <= 32 ? nvfp4::gemm_scratch_bytes(M, N, K) : 0;
-  l.zero = M <= 32 ? kLinearHeader + (nvfp4::gemm_zero_bytes(M, N, K) - 256) : kLinearHeader;
+  const size_t scratch = nvfp4::gemm_scratch_bytes(M, N, K);
+  l.zero = kLinearHeader + nvfp4::gemm_counter_bytes(M, N, K);
   l.x_codes = (kLinearHeader + scratch + 255) / 256 * 256;
   l.x_scales = l.x_codes + linear_codes_bytes(M, K);
   l.total = l.x_scales + nvfp4_scales_bytes(M, K, NVFP4_SF_SWIZZLED);

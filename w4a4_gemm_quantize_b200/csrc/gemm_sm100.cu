@@ -346,6 +346,117 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 // reads), and write BF16 through 128-byte-swizzled shared-memory boxes with TMA
 // stores.
 
+// The work of one CTA pair, as a sequence of items: an item is one 256 x 256 output tile
+// over a range of its K-tiles.  Tiles are done whole (data-parallel), except that, when
+// the tile count T is not a multiple of the pair count P and partial tiles are enabled,
+// the first P + T mod P tiles are done "stream-K": their K-tiles form one sequence of
+// units, tile-major, split evenly over the pairs, so that no pair idles through a last,
+// partial round.  A pair's stream-K range holds at least one tile's K-tiles, so a tile
+// is shared by at most two pairs: piece 0 (from K-tile 0) and piece 1 (up to the last
+// K-tile).  Both pieces store their FP32 partial tile in the slot of the later piece's
+// pair; the piece that finishes second sums the two, piece 0 plus piece 1, and writes C.
+// A pair does its pieces first, then its whole stream-K tiles, then its data-parallel
+// tiles, so that the sums overlap the remaining work.
+// Pair kernel: shapes it takes, and its shared-tile scratch -- a ticket counter and a
+// ready flag per slot, CTA and epilogue warp, then two pieces x two CTAs x 8 warps x
+// 32 x 128 FP32 per slot --
+// for up to kMaxPairSlots pairs (148 SMs); a larger grid runs without partial tiles.
+constexpr int kMaxPairSlots = 74;
+inline bool uses_pair_kernel(int64_t M, int64_t N) { return M > 128 && N > 128; }
+constexpr int kPairFlagOffset = kMaxPairSlots * 2 * 8;  // flags follow the counters (words)
+inline size_t pair_counter_bytes() { return (static_cast<size_t>(2 * kPairFlagOffset) * 4 + 255) / 256 * 256; }
+inline size_t pair_partial_bytes() { return static_cast<size_t>(kMaxPairSlots) * 2 * 2 * 8 * 32 * 128 * 4; }
+
+// Bounded wait for a flag that another CTA of the grid sets (every CTA of the pair
+// kernel is resident: one per SM, at most as many pairs as fit).
+__device__ __forceinline__ bool wait_flag(const uint32_t* flag, volatile uint32_t* abort, uint32_t* status,
+                                          uint32_t where) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (*reinterpret_cast<const volatile uint32_t*>(flag) != 0u) return true;
+    if ((n & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        *abort = 1u;
+        if (status) atomicCAS(status, 0u, where);
+        return false;
+      }
+    }
+  }
+}
+
+struct PairItem {
+  int tile;      // tile index, in tile_coords order
+  int kt0, kt1;  // K-tiles [kt0, kt1)
+  int slot;      // partial-tile slot of a shared tile; -1 for a whole tile
+  int piece;     // 0 or 1 for a shared tile
+};
+
+// Stream-K tiles (the first n_sk).  A shared tile costs its two pieces' epilogues
+// (the FP32 partial sums out, then in again while the accumulator is held) and the
+// stream-K part reads A and B with less reuse between neighbouring pairs; measured on
+// B200 this pays only when the last round would leave the pairs idle for at least ~40
+// K-tiles on average (e.g. K = 21504 with 672 tiles on 74 pairs, not K = 5376).
+__host__ __device__ __forceinline__ int pair_sk_tiles(int P, int T, int KT, bool partial_tiles) {
+  const int rem = T % P;
+  if (!partial_tiles || rem == 0 || T < P) return 0;
+  if (static_cast<int64_t>(P - rem) * KT < 40LL * P) return 0;
+  return P + rem;
+}
+
+__device__ __forceinline__ int pair_item_count(int pair, int P, int T, int KT, bool partial_tiles) {
+  const int n_sk = pair_sk_tiles(P, T, KT, partial_tiles);
+  const int64_t U = static_cast<int64_t>(n_sk) * KT;
+  const int64_t b0 = static_cast<int64_t>(pair) * U / P, b1 = static_cast<int64_t>(pair + 1) * U / P;
+  int n = 0;
+  if (n_sk > 0) n = static_cast<int>(b0 % KT != 0) + static_cast<int>(b1 % KT != 0) +
+                    static_cast<int>(b1 / KT - (b0 + KT - 1) / KT);
+  const int first = n_sk + pair;
+  return n + (first < T ? (T - first + P - 1) / P : 0);
+}
+
+// Item i of the pair: [start piece][end piece][whole stream-K tiles][data-parallel tiles].
+__device__ __forceinline__ PairItem pair_item(int i, int pair, int P, int T, int KT, bool partial_tiles) {
+  PairItem it;
+  it.slot = -1;
+  it.piece = 0;
+  it.kt0 = 0;
+  it.kt1 = KT;
+  const int n_sk = pair_sk_tiles(P, T, KT, partial_tiles);
+  if (n_sk > 0) {
+    const int64_t U = static_cast<int64_t>(n_sk) * KT;
+    const int64_t b0 = static_cast<int64_t>(pair) * U / P, b1 = static_cast<int64_t>(pair + 1) * U / P;
+    if (b0 % KT != 0) {
+      if (i == 0) {  // the end of a tile begun by the pair before
+        it.tile = static_cast<int>(b0 / KT);
+        it.kt0 = static_cast<int>(b0 % KT);
+        it.slot = pair;
+        it.piece = 1;
+        return it;
+      }
+      --i;
+    }
+    if (b1 % KT != 0) {
+      if (i == 0) {  // the start of a tile that the next pair finishes
+        it.tile = static_cast<int>(b1 / KT);
+        it.kt1 = static_cast<int>(b1 % KT);
+        it.slot = pair + 1;
+        it.piece = 0;
+        return it;
+      }
+      --i;
+    }
+    const int w0 = static_cast<int>((b0 + KT - 1) / KT), w1 = static_cast<int>(b1 / KT);
+    if (i < w1 - w0) {
+      it.tile = w0 + i;
+      return it;
+    }
+    i -= w1 - w0;
+  }
+  it.tile = n_sk + pair + i * P;
+  return it;
+}
+
 template <bool LR = false>
 struct PairCfg {
   static constexpr int BM = 128;                      // rows of A per CTA (256 per pair)
@@ -384,14 +495,15 @@ struct PairCfg {
   static_assert(BN + SF_REGIONS * SF_COLS <= TMEM_COLS, "TMEM budget");
 };
 
-template <bool LR, bool MX>
+template <bool LR, bool MX, bool SK = false>
 __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                      const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_lb,
                      const __grid_constant__ CUtensorMap tmap_thi, const __grid_constant__ CUtensorMap tmap_tlo,
                      int rank_lr, uint16_t* __restrict__ C, int64_t ldc, const float* __restrict__ a_gs,
-                     const float* __restrict__ b_gs, int M, int N, int K, uint32_t* __restrict__ status) {
+                     const float* __restrict__ b_gs, int M, int N, int K, uint32_t* __restrict__ status,
+                     uint32_t* __restrict__ piece_counters, float* __restrict__ piece_partials) {
   using Cfg = PairCfg<LR>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int R = Cfg::SF_REGIONS;
@@ -428,6 +540,10 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
   const int num_m = (M + 2 * Cfg::BM - 1) / (2 * Cfg::BM);
   const int num_n = (N + Cfg::BN - 1) / Cfg::BN;
   const int num_tiles = num_m * num_n;
+  // partial tiles (the stream-K part): a separate instantiation, launched when the
+  // schedule uses them (never with the low-rank branch, which adds its term once per tile)
+  const bool partial_tiles = SK && !LR && piece_partials != nullptr;
+  const int n_items = pair_item_count(pair, npairs, num_tiles, k_tiles, partial_tiles);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -479,9 +595,10 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
       for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
       int kc = 0, it = 0;
       bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += npairs, ++it) {
+      for (; it < n_items && ok; ++it) {
+        const PairItem item = pair_item(it, pair, npairs, num_tiles, k_tiles, partial_tiles);
         int tm, tn;
-        tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
+        tile_coords<Cfg::GROUP_M>(item.tile, num_m, num_n, tm, tn);
         if (LR) {
           // the tile's low-rank operands, once the previous tile's low-rank MMAs are done
           if (!mbar_wait_cluster(lora_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, status,
@@ -495,7 +612,7 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
           tma_load_2d_pair(sTH, &tmap_thi, lbar, 0, tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM);
           tma_load_2d_pair(sTL, &tmap_tlo, lbar, 0, tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM);
         }
-        for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+        for (int kt = item.kt0; kt < item.kt1; ++kt, ++kc) {
           const int s = kc % STAGES;
           const uint32_t ph = static_cast<uint32_t>(kc / STAGES) & 1u;
           if (!mbar_wait_cluster(&empty[s], ph ^ 1u, abort_flag, status, kErrWaitEmpty)) {
@@ -528,7 +645,8 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
       const uint32_t acc_full_own = smem_u32(acc_full);
       bool ok = true;
       int kc = 0, it = 0;
-      for (int t = pair; t < num_tiles && ok; t += npairs, ++it) {
+      for (; it < n_items && ok; ++it) {
+        const PairItem item = pair_item(it, pair, npairs, num_tiles, k_tiles, partial_tiles);
         if (!mbar_wait_cluster(acc_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, status,
                                kErrWaitAccEmpty)) {
           ok = false;
@@ -558,7 +676,7 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
           }
           tc_fence_after();
         }
-        for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+        for (int kt = item.kt0; kt < item.kt1; ++kt, ++kc) {
           const int s = kc % STAGES;
           const int r = s;
           // one wait per K-tile: the leader's scale warps arrive on sf_ready only after
@@ -576,10 +694,10 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
           for (int j = 0; j < na; ++j) {
             if constexpr (MX)
               mma_mxf4_block32_pair(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j),
-                                    idesc, t_sf + 4 * j, t_sf + 16 + 8 * j, (LR || (kt | j) != 0) ? 1u : 0u);
+                                    idesc, t_sf + 4 * j, t_sf + 16 + 8 * j, (LR || kt != item.kt0 || j != 0) ? 1u : 0u);
             else
               mma_mxf4nvf4_pair(t_acc, sdesc_kmajor_sw128(a_base + 32 * j), sdesc_kmajor_sw128(b_base + 32 * j),
-                                idesc, t_sf + 4 * j, t_sf + 16 + 8 * j, (LR || (kt | j) != 0) ? 1u : 0u);
+                                idesc, t_sf + 4 * j, t_sf + 16 + 8 * j, (LR || kt != item.kt0 || j != 0) ? 1u : 0u);
           }
           tc_commit_pair_both(smem_u32(&empty[s]));
         }
@@ -602,10 +720,11 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
       for (int s = 0; s < STAGES; ++s) issued_last[s] = -1;
       int kc = 0;
       bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += npairs) {
+      for (int it = 0; it < n_items && ok; ++it) {
+        const PairItem item = pair_item(it, pair, npairs, num_tiles, k_tiles, partial_tiles);
         int tm, tn;
-        tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
-        for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+        tile_coords<Cfg::GROUP_M>(item.tile, num_m, num_n, tm, tn);
+        for (int kt = item.kt0; kt < item.kt1; ++kt, ++kc) {
           const int s = kc % STAGES;
           if (kc >= STAGES && !mbar_wait(&sf_empty[s], (static_cast<uint32_t>(kc / STAGES) & 1u) ^ 1u, abort_flag,
                                          status, kErrWaitEmpty + 1)) {
@@ -633,8 +752,9 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
     const uint32_t sf_ready_leader0 = mapa_shared(smem_u32(&sf_ready[0]), 0u);
     int kc = 0, handled = 0;
     bool ok = true;
-    for (int t = pair; t < num_tiles && ok; t += npairs) {
-      for (int kt = 0; kt < k_tiles; ++kt, ++kc) {
+    for (int it = 0; it < n_items && ok; ++it) {
+      const PairItem item = pair_item(it, pair, npairs, num_tiles, k_tiles, partial_tiles);
+      for (int kt = item.kt0; kt < item.kt1; ++kt, ++kc) {
         if (kc % Cfg::SF_SETS != set) continue;
         const int s = kc % STAGES;
         const int r = s;
@@ -742,13 +862,118 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * HALF;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0u);
     uint8_t* box = sC + warp * Cfg::C_BOX_BYTES;
-    int it = 0;
     bool stored = false;
-    for (int t = pair; t < num_tiles; t += npairs, ++it) {
+    for (int it = 0; it < n_items; ++it) {
+      const PairItem item = pair_item(it, pair, npairs, num_tiles, k_tiles, partial_tiles);
       int tm, tn;
-      tile_coords<Cfg::GROUP_M>(t, num_m, num_n, tm, tn);
+      tile_coords<Cfg::GROUP_M>(item.tile, num_m, num_n, tm, tn);
       if (!warp_wait_cluster(acc_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, kErrWaitAccFull)) break;
       tc_fence_after();
+      // A shared tile (two pieces): the first piece to get here stores its FP32 partial
+      // sums and raises a flag; the second waits for the flag and adds them to its own,
+      // mine + other (FP32 addition commutes, so the sum does not depend on which piece
+      // came first), then writes C.  A warp's part is its 32 rows x 128 columns, stored
+      // as [column / 4][row][4] so that each store or load of the warp covers 512
+      // contiguous bytes; slot, piece, CTA and warp select the part.
+      constexpr size_t kPart = 32 * HALF;
+      const bool split = partial_tiles && item.slot >= 0;
+      bool first = false;
+      float* part = nullptr;  // the first piece: its own part; the second: the other's
+      const int entry = (item.slot * 2 + static_cast<int>(rank)) * 8 + warp;
+      if (split) {
+        uint32_t before = 0;
+        if (lane == 0) before = atomicAdd(&piece_counters[entry], 1u);
+        first = __shfl_sync(0xFFFFFFFFu, before, 0) == 0u;
+        const int pc = first ? item.piece : 1 - item.piece;
+        part = piece_partials + ((static_cast<size_t>(item.slot) * 2 + pc) * 2 + rank) * 8 * kPart +
+               static_cast<size_t>(warp) * kPart;
+        if (!first) {
+          bool got = true;
+          if (lane == 0) got = wait_flag(&piece_counters[kPairFlagOffset + entry], abort_flag, status, kErrWaitPiece);
+          if (!__shfl_sync(0xFFFFFFFFu, got, 0)) break;
+          __threadfence();
+        }
+      }
+      if (split && first) {
+#pragma unroll
+        for (int c = 0; c < HALF; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_lane + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<uint4*>(part + ((c / 4 + i) * 32 + lane) * 4) =
+                make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive(acc_empty);
+          else
+            mbar_arrive_cluster_relaxed(acc_empty_leader);
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicExch(&piece_counters[kPairFlagOffset + entry], 1u);
+        continue;
+      }
+      if (split) {
+        const int row0 = tm * 2 * Cfg::BM + static_cast<int>(rank) * Cfg::BM + quarter * 32;
+        const int col0 = tn * Cfg::BN + half * HALF;
+        // the second piece: 32 columns at a time, the other piece's sums loaded before the
+        // accumulator's (so that the loads overlap), summed, scaled, rounded to BF16 and
+        // staged as in the whole-tile store below
+#pragma unroll
+        for (int chunk = 0; chunk < 2; ++chunk) {
+          if (stored) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            const int c = chunk * 64 + sub * 32;
+            float4 o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = __ldcg(reinterpret_cast<const float4*>(part) + (c / 4 + i) * 32 + lane);
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(t_lane + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) {
+              const float4 x = o[2 * uu], y = o[2 * uu + 1];
+              const uint32_t* m = v + 8 * uu;
+              const uint4 w = make_uint4(
+                  pack_bf16x2(__fmul_rn(__fadd_rn(__uint_as_float(m[0]), x.x), alpha),
+                              __fmul_rn(__fadd_rn(__uint_as_float(m[1]), x.y), alpha)),
+                  pack_bf16x2(__fmul_rn(__fadd_rn(__uint_as_float(m[2]), x.z), alpha),
+                              __fmul_rn(__fadd_rn(__uint_as_float(m[3]), x.w), alpha)),
+                  pack_bf16x2(__fmul_rn(__fadd_rn(__uint_as_float(m[4]), y.x), alpha),
+                              __fmul_rn(__fadd_rn(__uint_as_float(m[5]), y.y), alpha)),
+                  pack_bf16x2(__fmul_rn(__fadd_rn(__uint_as_float(m[6]), y.z), alpha),
+                              __fmul_rn(__fadd_rn(__uint_as_float(m[7]), y.w), alpha)));
+              const int u = sub * 4 + uu;  // row `lane`, 16-byte unit u goes to u ^ (lane % 8)
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((u ^ (lane & 7)) << 4)) = w;
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < M && col0 + chunk * 64 < N) {
+            tma_store_2d(&tmap_c, box, col0 + chunk * 64, row0);
+            bulk_commit_group();
+          }
+          stored = true;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive(acc_empty);
+          else
+            mbar_arrive_cluster_relaxed(acc_empty_leader);
+        }
+        continue;
+      }
       uint32_t p[HALF / 2];
 #pragma unroll
       for (int c = 0; c < HALF; c += 32) {
@@ -805,8 +1030,8 @@ __global__ void __launch_bounds__(PairCfg<LR>::THREADS, 1)
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int q = chunk * 32 + 4 * u;
-          *reinterpret_cast<uint4*>(box + lane * 128 + ((u ^ (lane & 7)) << 4)) =
-              make_uint4(p[q], p[q + 1], p[q + 2], p[q + 3]);
+          const uint4 w = make_uint4(p[q], p[q + 1], p[q + 2], p[q + 3]);
+          *reinterpret_cast<uint4*>(box + lane * 128 + ((u ^ (lane & 7)) << 4)) = w;
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -1551,7 +1776,7 @@ bool encode_sf_map(CUtensorMap* map, const uint8_t* sf, int64_t rows, int64_t K,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool LR, bool MX>
+template <bool LR, bool MX, bool SK = false>
 int max_pair_clusters(int dev) {
   using Cfg = PairCfg<LR>;
   static std::once_flag once[64];
@@ -1569,9 +1794,9 @@ int max_pair_clusters(int dev) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaFuncSetAttribute(gemm_pair_kernel<LR, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemm_pair_kernel<LR, MX, SK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess ||
-        cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<LR, MX>, &cfg) != cudaSuccess) {
+        cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<LR, MX, SK>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       n = 0;
     }
@@ -1614,7 +1839,7 @@ template <bool LR, bool MX>
 cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gs, int64_t N, int64_t K,
                         uint16_t* c, int64_t ldc, uint32_t* status, const uint16_t* lora_b, const uint16_t* thi,
-                        const uint16_t* tlo, int64_t rank, cudaStream_t stream) {
+                        const uint16_t* tlo, int64_t rank, cudaStream_t stream, uint8_t* scratch = nullptr) {
   using Cfg = PairCfg<LR>;
   CUtensorMap ta, tb, tsa, tsb, tc, tlb, tth, ttl;
   if (!encode_codes_map(&ta, a_codes, M, K, 128) || !encode_codes_map(&tb, b_codes, N, K, 128) ||
@@ -1634,6 +1859,15 @@ cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float
   if (max_clusters <= 0) return cudaErrorLaunchOutOfResources;
   const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
   const int clusters = static_cast<int>(tiles < max_clusters ? tiles : max_clusters);
+  // partial tiles (the instantiation with the stream-K part) when the schedule uses them;
+  // they need the counters (cleared before the launch) and the partial-tile slots
+  const int k_tiles = static_cast<int>(((K + 63) / 64 + 3) / 4);
+  bool sk = false;
+  if constexpr (!LR && !MX)
+    sk = scratch != nullptr && clusters <= kMaxPairSlots &&
+         pair_sk_tiles(clusters, static_cast<int>(tiles), k_tiles, true) > 0 && max_pair_clusters<LR, MX, true>(dev) > 0;
+  uint32_t* piece_counters = sk ? reinterpret_cast<uint32_t*>(scratch) : nullptr;
+  float* piece_partials = sk ? reinterpret_cast<float*>(scratch + pair_counter_bytes()) : nullptr;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
   cfg.blockDim = dim3(Cfg::THREADS);
@@ -1647,8 +1881,15 @@ cudaError_t launch_pair(const uint8_t* a_codes, const uint8_t* a_sf, const float
   set_programmatic(attr[1]);
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  if constexpr (!LR && !MX) {
+    if (sk)
+      return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<LR, MX, true>, ta, tb, tsa, tsb, tc, tlb, tth, ttl,
+                                static_cast<int>(rank), c, ldc, a_gs, b_gs, static_cast<int>(M), static_cast<int>(N),
+                                static_cast<int>(K), status, piece_counters, piece_partials);
+  }
   return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<LR, MX>, ta, tb, tsa, tsb, tc, tlb, tth, ttl, static_cast<int>(rank), c,
-                            ldc, a_gs, b_gs, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), status);
+                            ldc, a_gs, b_gs, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), status,
+                            piece_counters, piece_partials);
 }
 
 // CTAs of the decode kernel: one per weight tile when the tiles number between 70 %
@@ -1739,19 +1980,30 @@ cudaError_t launch_tile(const CUtensorMap& ta, const CUtensorMap& tb, const uint
 
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K) {
   using Cfg = DecodeCfg<false>;
-  if (M > Cfg::BN) return 0;
-  // partial-tile slots for the largest grid the launcher uses (more CTAs, more segments)
-  const int64_t KT = (K + 255) / 256;
-  const int64_t T = (N + Cfg::BM - 1) / Cfg::BM;
-  const int64_t G = decode_grid(N, K, kMaxDecodeGrid);
-  const int64_t max_seg = decode_max_segments(KT, T * KT, G);
-  return decode_counter_bytes(N) + static_cast<size_t>(T * max_seg) * Cfg::BM * Cfg::BN * 4;
+  if (M <= Cfg::BN) {
+    // partial-tile slots for the largest grid the launcher uses (more CTAs, more segments)
+    const int64_t KT = (K + 255) / 256;
+    const int64_t T = (N + Cfg::BM - 1) / Cfg::BM;
+    const int64_t G = decode_grid(N, K, kMaxDecodeGrid);
+    const int64_t max_seg = decode_max_segments(KT, T * KT, G);
+    return decode_counter_bytes(N) + static_cast<size_t>(T * max_seg) * Cfg::BM * Cfg::BN * 4;
+  }
+  if (uses_pair_kernel(M, N)) return pair_counter_bytes() + pair_partial_bytes();
+  return 0;
 }
 
-size_t gemm_zero_bytes(int64_t M, int64_t N, int64_t) {
+size_t gemm_counter_bytes(int64_t M, int64_t N, int64_t) {
+  if (M <= DecodeCfg<false>::BN) return decode_counter_bytes(N);
+  if (uses_pair_kernel(M, N)) return pair_counter_bytes();
+  return 0;
+}
+
+size_t gemm_zero_bytes(int64_t M, int64_t N, int64_t K) {
   // the status word of every kernel (a clear inside the kernel could erase the
-  // timeout code of a CTA that started earlier), plus the decode kernel's tile counters
-  return M <= DecodeCfg<false>::BN ? 256 + decode_counter_bytes(N) : sizeof(uint32_t);
+  // timeout code of a CTA that started earlier), plus the counters at the start of the
+  // scratch that follows it (decode tiles, or the pair kernel's shared tiles)
+  const size_t counters = gemm_counter_bytes(M, N, K);
+  return counters > 0 ? 256 + counters : sizeof(uint32_t);
 }
 
 cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs, int64_t M,
@@ -1765,9 +2017,9 @@ cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
     return launch_decode<false, false>(tw, tx, tw, tw, tw, 0, a_sf, a_gs, nullptr, 0, nullptr, nullptr, M, b_sf, b_gs,
                                        N, K, c, ldc, status, scratch, stream);
   }
-  if (M > 128 && N > 128)
+  if (uses_pair_kernel(M, N))
     return launch_pair<false, false>(a_codes, a_sf, a_gs, M, b_codes, b_sf, b_gs, N, K, c, ldc, status, nullptr, nullptr,
-                              nullptr, 0, stream);
+                                     nullptr, 0, stream, scratch ? scratch : reinterpret_cast<uint8_t*>(status) + 256);
   const int bn = N > 128 ? 256 : 128;
   CUtensorMap ta, tb;
   if (!encode_codes_map(&ta, a_codes, M, K, 128) || !encode_codes_map(&tb, b_codes, N, K, bn))

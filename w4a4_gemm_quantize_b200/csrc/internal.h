@@ -83,14 +83,18 @@ cudaError_t launch_lora_down(const uint16_t* x, int64_t M, int64_t K, int64_t ld
 size_t lora_partial_bytes(int64_t M, int64_t K, int64_t R);
 size_t lora_counter_bytes(int64_t M);
 
-// Bytes the GEMM needs in its workspace after the 256-byte status block
-// (split-K partial tiles of the small-M kernel); 0 when none.
+// Bytes the GEMM needs in its workspace after the 256-byte status block: the
+// small-M kernel's tile counters and split partial tiles, or the pair kernel's
+// shared-tile counters and partial tiles; 0 when none.
 size_t gemm_scratch_bytes(int64_t M, int64_t N, int64_t K);
 
 // Bytes at the start of the workspace that must be zero when the GEMM launches
-// (cleared with one memset before the kernel): the status word, and for M <= 32
-// the decode kernel's tile counters after the 256-byte status block.
+// (cleared with one memset before the kernel): the status word, and the counters at
+// the start of the scratch after the 256-byte status block.
 size_t gemm_zero_bytes(int64_t M, int64_t N, int64_t K);
+
+// The counter bytes at the start of the GEMM scratch (0 when none).
+size_t gemm_counter_bytes(int64_t M, int64_t N, int64_t K);
 
 // Number of kernel launches the last call of each entry point enqueued (for
 // the benchmark's launch count); host-side bookkeeping only.

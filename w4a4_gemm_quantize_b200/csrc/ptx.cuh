@@ -23,6 +23,7 @@ enum : uint32_t {
   kErrWaitDrain = 0x500,     // teardown waiting for in-flight copies / MMAs
   kErrSelfTest = 0x600,      // the wait of nvfp4_selftest_wait_timeout (expected to give up)
   kErrLora = 0x700,          // the low-rank down-projection kernel (plus the wait's own code)
+  kErrWaitPiece = 0x800,     // epilogue waiting for the other piece of a shared tile
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
