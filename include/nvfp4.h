@@ -93,7 +93,9 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t cols);
  *   layout       layout of `scales`.
  *   global_scale_in  device float or NULL.  NULL: s_g = amax(|x|) / 2688 (an
  *                all-zero tensor gets 1.0), computed on the device by a first
- *                pass over x.  Non-NULL: use *global_scale_in (> 0) and skip
+ *                pass over x -- for an ABSMAX tensor of at most 262144 elements
+ *                inside the quantizing launch itself (one cluster of CTAs), the
+ *                same value.  Non-NULL: use *global_scale_in (> 0) and skip
  *                that pass.
  *   codes        device, nvfp4_codes_bytes(rows, cols) bytes, dense (row stride cols/2).
  *   scales       device, nvfp4_scales_bytes(rows, cols, layout) bytes; every byte
@@ -171,8 +173,8 @@ size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *                section 2, the third of the "three questions" every quantization
  *                scheme answers -- activation scales come from calibration on real
  *                activations), nothing reads the whole of x first.  NULL:
- *                s_g = amax(|x|) / 2688 computed on the device by a first pass, as
- *                nvfp4_quantize does.
+ *                s_g = amax(|x|) / 2688 computed on the device as nvfp4_quantize
+ *                does (for M x K <= 262144 inside the quantizing launch).
  *   w_codes, w_scales, w_global_scale  the weight N x K as nvfp4_quantize writes it
  *                (scales SWIZZLED).
  *   c            device BF16, M x N, row stride ldc (ldc >= N, ldc % 8 == 0).

@@ -124,6 +124,13 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
 
   const bool swz = layout == NVFP4_SF_SWIZZLED;
   uint32_t* amax_word = static_cast<uint32_t*>(workspace);
+  if (global_scale_in == nullptr && rows > 0 && cols > 0 && nvfp4::quantize_fuses_amax(rows, cols, mode)) {
+    // a small tensor: one launch computes the amax and encodes
+    st = from_cuda(nvfp4::launch_quantize_fused(static_cast<const uint16_t*>(x), rows, cols, ld_x, swz, codes,
+                                                scales, global_scale_out, block_err, s));
+    if (st == NVFP4_OK) ++nvfp4::g_last_launches;
+    return st;
+  }
   if (global_scale_in == nullptr) {
     if (cudaMemsetAsync(amax_word, 0, sizeof(uint32_t), s) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (rows > 0 && cols > 0) {
@@ -267,7 +274,9 @@ nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, int64_t ld_x, con
   // tile counters, so that the kernels after it follow one another with programmatic
   // dependent launch
   if (cudaMemsetAsync(ws, 0, l.zero, s) != cudaSuccess) return NVFP4_ERR_CUDA;
-  if (x_global_scale == nullptr) {
+  // a small activation without a given s_g: one launch computes its amax and encodes it
+  const bool fused_amax = x_global_scale == nullptr && nvfp4::quantize_fuses_amax(M, K, NVFP4_SCALE_ABSMAX);
+  if (x_global_scale == nullptr && !fused_amax) {
     st = from_cuda(nvfp4::launch_amax(xb, M, K, ld_x, amax_word, s));
     if (st != NVFP4_OK) return st;
     ++nvfp4::g_last_launches;
@@ -275,8 +284,9 @@ nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, int64_t ld_x, con
   uint8_t* a_codes = ws + l.x_codes;
   uint8_t* a_scales = ws + l.x_scales;
   float* a_gs = x_global_scale ? nullptr : reinterpret_cast<float*>(ws + 260);
-  st = from_cuda(nvfp4::launch_quantize(xb, M, K, ld_x, NVFP4_SCALE_ABSMAX, true, x_global_scale, amax_word, a_codes,
-                                        a_scales, a_gs, nullptr, s));
+  st = from_cuda(fused_amax ? nvfp4::launch_quantize_fused(xb, M, K, ld_x, true, a_codes, a_scales, a_gs, nullptr, s)
+                            : nvfp4::launch_quantize(xb, M, K, ld_x, NVFP4_SCALE_ABSMAX, true, x_global_scale,
+                                                     amax_word, a_codes, a_scales, a_gs, nullptr, s));
   if (st != NVFP4_OK) return st;
   ++nvfp4::g_last_launches;
   st = from_cuda(nvfp4::launch_gemm(a_codes, a_scales, x_global_scale ? x_global_scale : a_gs, M, w_codes, w_scales,

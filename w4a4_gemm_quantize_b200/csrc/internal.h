@@ -19,6 +19,12 @@ nvfp4_status validate_quantize(const void* x, int64_t rows, int64_t cols, int64_
 // API layer has already validated.
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax_bits,
                         cudaStream_t stream);
+// Absmax quantization of a small tensor (quantize_fuses_amax) in one launch that also
+// computes the amax: s_g = amax / 2688 by the same rule as the two-pass path.
+bool quantize_fuses_amax(int64_t rows, int64_t cols, int mode);
+cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, bool swizzled,
+                                  uint8_t* codes, uint8_t* scales, float* gs_out, float* block_err,
+                                  cudaStream_t stream);
 cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int mode,
                             bool swizzled, const float* gs_in, const uint32_t* amax_bits, uint8_t* codes,
                             uint8_t* scales, float* gs_out, float* block_err, cudaStream_t stream);

@@ -40,6 +40,10 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kThreads = 256;
+// CTAs (one cluster) of the quantizer that computes the amax itself; used for tensors of
+// at most kFusedMaxElems elements, where the separate amax pass is mostly launch cost.
+constexpr int kFusedCtas = 8;
+constexpr int64_t kFusedMaxElems = 256 * 1024;
 
 // Streaming 16-byte load: read-only path, no L1 allocation, 256-byte L2 fetches.
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
@@ -199,7 +203,11 @@ __device__ __forceinline__ void mse_walk(const uint64_t (&x2)[8], float amax_b, 
 // One warp handles 32 consecutive blocks of one row (lane = block); warps walk a
 // fixed column chunk down the rows, so block coordinates and output offsets need
 // no division.
-template <int MODE, bool SWZ>
+// FUSED: the tensor's amax is computed by the launch itself -- one cluster of
+// kFusedCtas CTAs, each CTA's maximum in shared memory, combined over the cluster
+// through distributed shared memory -- so a small tensor needs neither the amax pass
+// nor its cleared word (s_g from the same rule and arithmetic as the two-pass path).
+template <int MODE, bool SWZ, bool FUSED = false>
 __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, const float* __restrict__ gs_in,
     const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
@@ -215,10 +223,42 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(
   constexpr int kRing = MODE == 1 ? 64 : 1;
   __shared__ uint4 ring[3][kThreads / 32][kRing];
   grid_dependents_launch();  // the GEMM behind this pass may set up and start its weight stream
-  grid_dependency_wait();    // launched behind the amax pass (programmatic launch)
+  grid_dependency_wait();    // launched behind the amax pass or the producer of x (programmatic launch)
   const int64_t nblk = cols / 16;
   const int64_t atoms_per_group = (nblk + 3) / 4;
-  const float sg = global_scale(gs_in, amax_bits);
+  float sg;
+  if constexpr (FUSED) {
+    __shared__ uint32_t cta_max;
+    uint32_t m = 0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t vpr = cols / 8, nvec = rows * vpr;
+    if (ld == cols) {
+      for (int64_t i = tid; i < nvec; i += stride) m = vmax_mag(m, ld_nc_v4(x + i * 8));
+    } else {
+      for (int64_t i = tid; i < nvec; i += stride) {
+        const int64_t r = i / vpr, c = i - r * vpr;
+        m = vmax_mag(m, ld_nc_v4(x + r * ld + c * 8));
+      }
+    }
+    m = __reduce_max_sync(0xFFFFFFFFu, max(m & 0xFFFFu, m >> 16));
+    __shared__ uint32_t warp_max[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      m = threadIdx.x < kThreads / 32 ? warp_max[threadIdx.x] : 0u;
+      m = __reduce_max_sync(0xFFFFFFFFu, m);
+      if (threadIdx.x == 0) cta_max = m;
+    }
+    cluster_sync();  // every CTA's maximum is in its shared memory
+    uint32_t g = 0;
+    for (uint32_t r = 0; r < static_cast<uint32_t>(kFusedCtas); ++r)
+      g = max(g, ld_shared_cluster_u32(mapa_shared(smem_u32(&cta_max), r)));
+    cluster_sync();  // no CTA leaves while another still reads its word
+    sg = global_scale(nullptr, &g);
+  } else {
+    sg = global_scale(gs_in, amax_bits);
+  }
   if (gs_out && blockIdx.x == 0 && threadIdx.x == 0) *gs_out = sg;
   const float d6 = __fmul_rn(6.0f, sg);
   if (threadIdx.x < 128) {
@@ -616,6 +656,36 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64
   else
     e = swizzled ? NVFP4_Q(0, true) : NVFP4_Q(0, false);
 #undef NVFP4_Q
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+bool quantize_fuses_amax(int64_t rows, int64_t cols, int mode) {
+  return mode == 0 && rows * cols <= kFusedMaxElems;
+}
+
+cudaError_t launch_quantize_fused(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, bool swizzled,
+                                  uint8_t* codes, uint8_t* scales, float* gs_out, float* block_err,
+                                  cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kFusedCtas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kFusedCtas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e =
+      swizzled ? cudaLaunchKernelEx(&cfg, quantize_kernel<0, true, true>, x, rows, cols, ld,
+                                    static_cast<const float*>(nullptr), static_cast<const uint32_t*>(nullptr), codes,
+                                    scales, gs_out, block_err)
+               : cudaLaunchKernelEx(&cfg, quantize_kernel<0, false, true>, x, rows, cols, ld,
+                                    static_cast<const float*>(nullptr), static_cast<const uint32_t*>(nullptr), codes,
+                                    scales, gs_out, block_err);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
