@@ -7,10 +7,10 @@
 // tensors and are applied per block inside the kernel; the result is BF16.
 //
 // Three kernels, chosen by launch_gemm from the shape: gemm_pair_kernel (M > 128
-// and N > 128: CTA pairs on 256 x 256 tiles), gemm_decode_kernel (M <= 32: the
-// weight stream split evenly over the SMs) and gemm_kernel<BN> (the other shapes),
-// each described where it is defined.  All are launched with programmatic
-// dependent launch.
+// and N > 128: CTA pairs on 256 x 256 tiles, with a stream-K instantiation for the
+// last round of long-K shapes), gemm_decode_kernel (M <= 32: the weight stream
+// split evenly over the SMs) and gemm_kernel<BN> (the other shapes), each described
+// where it is defined.  All are launched with programmatic dependent launch.
 //
 // gemm_kernel<BN>: a persistent kernel, one CTA per SM, each CTA walking 128 x BN output
 // tiles in a grouped order (GROUP_M row-tiles at a time, so the CTAs running at

@@ -26,9 +26,11 @@
 // per 16-value block (2 x 128-bit loads, packed 8-byte code stores), one warp per
 // 32 consecutive blocks of a row, per-CTA tables of the decoded scales and their
 // reciprocals, hardware cvt for E4M3 and E2M1 rounding, swizzled scale bytes
-// stored four at a time; the encode kernel also zeroes the swizzled padding.
-// Every kernel is launched with programmatic dependent launch and waits for its
-// predecessor before reading its inputs.
+// stored four at a time; the encode kernel also zeroes the swizzled padding.  The
+// MSE search queues the blocks whose walk goes past f = 0.9 per warp and resumes
+// them 32 at a time; a small absmax tensor computes its amax inside the encode
+// launch (one cluster).  Every kernel is launched with programmatic dependent launch
+// and waits for its predecessor before reading its inputs.
 #include <cuda_runtime.h>
 
 #include "internal.h"
