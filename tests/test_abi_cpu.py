@@ -231,6 +231,13 @@ def test_linear_workspace_layout(lib):
         act = -(-(M * 2048) // 256) * 256 + lib.nvfp4_scales_bytes(M, 4096, 0)
         assert lib.nvfp4_linear_workspace_bytes(M, 14336, 4096) >= 512 + gemm_scratch + act
     assert lib.nvfp4_linear_workspace_bytes(4096, 14336, 4096) >= 512 + 4096 * 2048 + 4096 * 256
+    # M, N > 128: the CTA-pair GEMM's shared-tile counters and partial tiles come before the
+    # activation's codes and scales
+    for (M, N, K) in [(4096, 14336, 4096), (8192, 5376, 21504)]:
+        gemm_scratch = lib.nvfp4_gemm_workspace_bytes(M, N, K) - 256
+        act = -(-(M * K // 2) // 256) * 256 + lib.nvfp4_scales_bytes(M, K, 0)
+        assert gemm_scratch > 38_000_000
+        assert lib.nvfp4_linear_workspace_bytes(M, N, K) >= 512 + gemm_scratch + act
 
 
 def test_linear_lora_validation_before_any_cuda_call(lib):
